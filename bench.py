@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of relative-bias GQA decode attention on B200.
+
+One step = one layer-call of the whole hot path (split plan, partial kernel,
+LSE-merge combine) over one batch of synthetic inputs already resident in
+HBM.  Default workload: batch 1, 1 decode token, 48 query / 8 KV heads,
+head dim 128, full attention over a 100,000-token paged bf16 cache (64-token
+pages in random order), relative table NB = 1,280 (1,024 exact + 256 log
+buckets to 2^20).  The L2 cache is flushed (a 2 x L2-size write) before every
+timed step; only the attention kernels sit between the CUDA events.
+
+Prints one JSON line (rank 0).  `value` is achieved HBM throughput in GB/s
+(algorithmic bytes: every visible K/V row once, every needed relative-table
+row once, q/out/lse), aggregated over all ranks; `us_per_call` is the mean
+device time per layer-call.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle as the baseline arm
+Under torchrun every rank runs its own replica of the workload (independent
+problems, no collective on the data path): weak scaling.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("µs/layer and achieved HBM GB/s (% of roofline), "
+          "48/8-head d128 decode @100K ctx")
+DEFAULT_WORKLOAD = "full_100k"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ("relative_bias_gqa_b200/csrc/rel_attn_kernels.cuh",
+                  "relative_bias_gqa_b200/csrc/sm100_ptx.cuh",
+                  "relative_bias_gqa_b200/csrc/rel_attn.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "partial_kernel_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------ bookkeeping
+def algorithmic_bytes(case, bucket_fn, out_bytes=2):
+    """Bytes the call must move: visible K/V rows once, the relative-table
+    rows [0, bucket(max distance)] of every KV head once, q, out, lse, the
+    block-table entries read and seq_lens."""
+    lens = case.seq_lens.cpu().tolist()
+    T, Hq, Hkv, D, P = (case.q_tokens, case.num_q_heads, case.num_kv_heads,
+                        case.head_dim, case.page_size)
+    W = case.window
+    kv = 0
+    pages = 0
+    d_max = 0
+    for L in lens:
+        lo = max(0, L - T - W + 1) if W > 0 else 0
+        kv += (L - lo) * Hkv * D * 2 * 2
+        pages += (L - 1) // P - lo // P + 1
+        d_max = max(d_max, min(W - 1, L - 1) if W > 0 else L - 1)
+    r_rows = bucket_fn(d_max) + 1
+    rel = r_rows * Hkv * D * 2
+    small = len(lens) * T * Hq * (D * 2 + D * out_bytes + 4) + pages * 4 + len(lens) * 4
+    return kv + rel + small, dict(kv=kv, rel=rel, other=small)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, samples = [], None, set(), 0
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            samples += 1
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [x for x in sm if mx and x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": samples}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(src_hash):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_hash") != src_hash:
+        return None
+    return t.get("dram_bytes_per_launch_full_size")
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_throughput(case, seconds: float, kv_heads: int = 1):
+    """The fp64 oracle, as it stands, on KV head 0 of the workload (its G
+    query heads over the whole visible context), repeated for ~`seconds`."""
+    import numpy as np
+    import oracle
+    G = case.num_q_heads // case.num_kv_heads
+    idx = case.block_table[0].long()
+    L = int(case.seq_lens[0])
+    n_pages = math.ceil(L / case.page_size)
+    pages = idx[:n_pages]
+    sub_k = case.k_cache[pages][:, :kv_heads].cpu()
+    sub_v = case.v_cache[pages][:, :kv_heads].cpu()
+    bt = torch_arange_row(n_pages)
+    q = case.q[:1, :, :G * kv_heads].cpu()
+    rel = case.rel_table[:kv_heads].cpu()
+    sl = case.seq_lens[:1].cpu()
+    W = case.window
+    lo = max(0, L - case.q_tokens - W + 1) if W > 0 else 0
+    nbytes = (L - lo) * kv_heads * 128 * 4
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        oracle.rel_attn_decode_ref(q, sub_k, sub_v, bt, sl, rel, W)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    cores = len(os.sched_getaffinity(0))
+    return {"value": calls * nbytes / el / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": (f"KV head 0 of {case.name} ({G} query heads, {L - lo} visible keys), "
+                       f"{calls} calls in {el:.1f} s; numpy fp64 with up to {cores} BLAS threads"),
+            "seconds": el}
+
+
+def torch_arange_row(n):
+    import torch
+    return torch.arange(n, dtype=torch.int32)[None]
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from relative_bias_gqa_b200 import rel_attn, workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    case = workloads.make_workload(args.workload, seed=args.seed + rank, device=dev)
+    prep = rel_attn.Prepared(case.q, case.k_cache, case.v_cache, case.block_table, case.seq_lens,
+                             case.rel_table, case.window, args.num_splits,
+                             max_seq_len=case.max_seq_len, out_fp32=False)
+    S = prep.num_splits
+    bucket = lambda d: rel_attn.rel_attn_bucket(prep.shape, d)
+    nbytes, parts = algorithmic_bytes(case, bucket)
+    props = torch.cuda.get_device_properties(dev)
+    flush = torch.empty(2 * max(props.L2_cache_size, 64 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        prep.partial()
+        prep.combine()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if prep.workspace.read_status() != rel_attn.REL_ATTN_OK:
+        raise RuntimeError("device status error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    # A short device-side sleep after the flush keeps the GPU busy while the
+    # host submits the step, so the events bracket device execution only.
+    sleep_cycles = 200_000
+    for i in range(K):
+        flush.zero_()
+        torch.cuda._sleep(sleep_cycles)
+        ev[i][0].record(stream)
+        prep.partial()
+        ev[i][1].record(stream)
+        prep.combine()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    t_step = [e[0].elapsed_time(e[2]) for e in ev]
+    t_part = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = sum(t_step)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    status = prep.workspace.read_status()
+
+    # the fused entry point (partial + PDL-chained combine in one call)
+    Kf = min(K, 2000)
+    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kf)]
+    for i in range(Kf):
+        flush.zero_()
+        torch.cuda._sleep(sleep_cycles)
+        evf[i][0].record(stream)
+        prep.decode()
+        evf[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_fused = [e[0].elapsed_time(e[1]) for e in evf]
+
+    # end to end: host q / block table / seq_lens in, host out / lse back
+    h_q = case.q.cpu().pin_memory()
+    h_bt = case.block_table.cpu().pin_memory()
+    h_sl = case.seq_lens.cpu().pin_memory()
+    h_out = torch.empty(prep.out.shape, dtype=prep.out.dtype).pin_memory()
+    h_lse = torch.empty(prep.lse.shape, dtype=prep.lse.dtype).pin_memory()
+    Ke = min(K, 2000)
+    eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+    for i in range(Ke):
+        flush.zero_()
+        eve[i][0].record(stream)
+        case.q.copy_(h_q, non_blocking=True)
+        case.block_table.copy_(h_bt, non_blocking=True)
+        case.seq_lens.copy_(h_sl, non_blocking=True)
+        prep.decode()
+        h_out.copy_(prep.out, non_blocking=True)
+        h_lse.copy_(prep.lse, non_blocking=True)
+        eve[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = [e[0].elapsed_time(e[1]) for e in eve]
+    h2d = h_q.numel() * 2 + h_bt.numel() * 4 + h_sl.numel() * 4
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        mean_step = total_ms / K
+        mean_part = statistics.fmean(t_part)
+        achieved = nbytes / (mean_part * 1e-3) / 1e9
+        value = world * K * nbytes / (total_ms * 1e-3) / 1e9
+        src_hash = kernel_source_hash()
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = oracle_throughput(case, args.cpu_seconds)
+        e2e_gbs = world * nbytes / (statistics.fmean(t_e2e) * 1e-3) / 1e9
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(mean_step, 6),
+            "us_per_call": round(mean_step * 1e3, 2),
+            "us_per_call_p10_p50_p90": [round(x * 1e3, 2) for x in
+                                        statistics.quantiles(t_step, n=10)[0:9:4]],
+            "us_per_call_fused": round(statistics.fmean(t_fused) * 1e3, 2),
+            "us_partial_kernel": round(mean_part * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) relative table)",
+            "config": {"workload": args.workload, "batch": case.batch, "q_tokens": case.q_tokens,
+                       "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
+                       "head_dim": case.head_dim, "seq_lens_max": case.max_seq_len,
+                       "window": case.window, "num_buckets": case.num_buckets,
+                       "page_size": case.page_size, "num_splits": S,
+                       "algorithmic_bytes_per_call": nbytes, "bytes_breakdown": parts,
+                       "l2": "flushed before every timed step (2 x L2 write)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                         else "fallback 6.65 TB/s",
+                         "kernel": "rel_attn_partial_kernel",
+                         "traffic": load_traffic(src_hash),
+                         "frac_of_8TBps_nominal": round(achieved / 8000.0, 4)},
+            "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
+                    "us_per_call": round(statistics.fmean(t_e2e) * 1e3, 2),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "q, block table and seq_lens copied in from pinned host memory and "
+                            "out + lse copied back inside each timed step; the KV cache and "
+                            "relative table are resident model state"},
+            "gpu_launches": K * (2 if S > 1 else 1),
+            "clocks": clocks,
+            "device_status": rel_attn.error_string(status),
+            "kernel_source_hash": src_hash,
+            "library": rel_attn.version(),
+        }
+        if cpu is not None:
+            result["cpu_baseline"] = cpu
+    return result
+
+
+# ----------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle timed on this host's cores, as the baseline arm."""
+    if rank != 0:
+        return None
+    import torch
+    from relative_bias_gqa_b200 import workloads
+    import oracle
+    case = workloads.make_workload(args.workload, seed=args.seed, device="cpu")
+    G = case.num_q_heads // case.num_kv_heads
+    L = int(case.seq_lens[0])
+    W = case.window
+    budget = 150.0 / max(1, args.steps + args.warmup)        # seconds per step
+    # a bounded sample: KV head 0, the last n visible keys of sequence 0,
+    # at their true positions (so the log buckets are exercised)
+    lo = max(0, L - case.q_tokens - W + 1) if W > 0 else 0
+    P = case.page_size
+    first = lo // P
+    n_pages_all = (L - 1) // P - first + 1
+    pages = case.block_table[0, first:first + n_pages_all].long()
+    k_all = case.k_cache[pages][:, :1].float().numpy()
+    v_all = case.v_cache[pages][:, :1].float().numpy()
+    q = case.q[0, :, :G].float().numpy()
+    rel = case.rel_table[0].float().numpy()
+    key_pos_all = __import__("numpy").arange(first * P, first * P + n_pages_all * P)
+    keep = (key_pos_all >= lo) & (key_pos_all < L)
+    keys = k_all.reshape(-1, 128)[keep]
+    vals = v_all.reshape(-1, 128)[keep]
+    key_pos = key_pos_all[keep]
+    q_pos = L - case.q_tokens + __import__("numpy").arange(case.q_tokens)
+
+    def one(n):
+        oracle.attend_at_positions(q, q_pos, keys[-n:], vals[-n:], key_pos[-n:], rel, W,
+                                   case.num_buckets)
+
+    n = min(len(keys), 4096)
+    t0 = time.perf_counter()
+    one(n)
+    dt = time.perf_counter() - t0
+    n = int(max(1024, min(len(keys), n * budget / max(dt, 1e-6))))
+    for _ in range(args.warmup):
+        one(n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one(n)
+    el = time.perf_counter() - t0
+    nbytes = n * 128 * 2 * 2
+    value = args.steps * nbytes / el / 1e9
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"KV head 0 of {args.workload}: the last {n} visible keys at their true positions, "
+              f"{case.q_tokens} token(s) x {G} query heads per step (fp64 numpy oracle)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    dist_init = False
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        dist_init = True
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist_init:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

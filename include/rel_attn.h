@@ -1,0 +1,164 @@
+/*
+ * rel_attn.h -- C ABI of the B200 (sm_100a) relative-bias GQA decode library.
+ *
+ * One operation: decode-time grouped-query attention over a paged bf16 KV
+ * cache with a learned relative-position term added to the pre-softmax
+ * logits.  For query token t of sequence b (position p = L_b - T + t) and
+ * query head hq (KV head h = hq / (Hq/Hkv)):
+ *
+ *   s_j = ( q.k_j + q.R_h[bucket(p - j)] ) / sqrt(D),   j in J_t
+ *   J_t = { j : 0 <= j <= p,  and p - j <= W - 1 when W > 0 }
+ *   lse = ln sum_j exp(s_j),   out = sum_j exp(s_j - lse) v_j
+ *
+ * bucket(d): d for d < E (E = exact_buckets, 1024); beyond that NL = NB - E
+ * log-spaced buckets with lower edges e_k = ceil(E (Dmax/E)^(k/NL)),
+ * bucket = E + min(NL-1, max{k : e_k <= d}); when NB <= E, min(d, NB-1).
+ *
+ * Sources: "vLLM TML Inkling 지원", section "TML Inkling 모델 아키텍처"
+ * (learned relative term added to the pre-softmax logits instead of RoPE;
+ * GQA with head size 128); "vLLM、Inkling 2 Smallを初日サポート GB200で630
+ * tok/s", section "モデルの構成" (48 query / 8 KV heads, sliding window
+ * 1,024) and section "vLLMの最適化と性能" (the GQA group's 6 heads packed into
+ * one 64-row tile of a decode kernel); "vLLM TML Inkling 지원", section
+ * "저지연 컬렉티브 및 커널" (sheared relative bias; num_splits chosen from
+ * batch size and KV length).  The pages give no formula: the form and the
+ * bucket function above are this library's reading.
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them.  Host-side arguments are the
+ *     shape struct and scalars.
+ *   - Return value 0 on success, a negative REL_ATTN_ERR_* code otherwise.
+ *     Arguments are validated before anything is launched: on an error
+ *     nothing runs on the stream.
+ *   - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The caller synchronises.
+ *   - One workspace must not be used by two calls that run concurrently.
+ */
+#ifndef REL_ATTN_H
+#define REL_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define REL_ATTN_OK                       0
+#define REL_ATTN_ERR_INVALID_ARG         -1  /* bad pointer, shape or scalar      */
+#define REL_ATTN_ERR_WORKSPACE_TOO_SMALL -2  /* workspace_bytes below the query  */
+#define REL_ATTN_ERR_CUDA                -3  /* CUDA runtime / launch failure     */
+#define REL_ATTN_ERR_TIMEOUT             -4  /* a device-side bounded wait expired */
+#define REL_ATTN_ERR_BAD_SEQ             -5  /* device saw seq_len or page out of range */
+#define REL_ATTN_ERR_NO_DEVICE           -6  /* current device is not sm_100     */
+
+/* Problem shape.  All fields are host integers. */
+typedef struct rel_attn_shape {
+  int batch;             /* B >= 1                                              */
+  int q_tokens;          /* T, query tokens per sequence, 1..8 (verify steps)  */
+  int num_q_heads;       /* Hq                                                  */
+  int num_kv_heads;      /* Hkv, Hq % Hkv == 0, G = Hq/Hkv == 6, G*T <= 48      */
+  int head_dim;          /* D, must be 128                                      */
+  int page_size;         /* P, must be 64                                       */
+  int num_pages;         /* pages in the K/V pool                               */
+  int max_pages_per_seq; /* row stride (in entries) of block_table             */
+  int num_buckets;       /* NB, rows of each KV head's relative table          */
+  int exact_buckets;     /* E (1024); 1 <= E                                    */
+  int max_distance;      /* Dmax (2^20); E < Dmax                               */
+  int max_seq_len;       /* host upper bound on seq_lens (0: use the block-table
+                            capacity); used only by the split heuristic        */
+  int out_fp32;          /* 0: out is bf16, 1: out is fp32                     */
+} rel_attn_shape;
+
+/*
+ * rel_attn_decode -- the whole hot path: split-KV partial kernel, then (when
+ * num_splits > 1) the LSE-merge combine kernel.
+ *
+ *   q           bf16 [B, T, Hq, D], row-major.
+ *   k_cache     bf16 [num_pages, Hkv, P, D]: one (page, KV head) is a
+ *   v_cache     contiguous P x D block.  16-byte aligned.
+ *   block_table int32 [B, max_pages_per_seq]: physical page of logical page
+ *               i of sequence b.  Only entries that hold keys some query
+ *               token can see are read (others may be anything, e.g. -1).
+ *   seq_lens    int32 [B]: context length L_b including the T query tokens;
+ *               T <= L_b <= max_pages_per_seq * P.  Device memory.
+ *   rel_table   bf16 [Hkv, NB, D]: relative embeddings R_h.  16-byte aligned.
+ *   window      W > 0: sliding window of W keys (self included); W <= 0: full.
+ *   num_splits  KV splits per (sequence, KV head), 1..256; <= 0 picks the
+ *               heuristic (rel_attn_choose_splits).
+ *   out         [B, T, Hq, D], bf16 or fp32 per shape->out_fp32.
+ *   lse         fp32 [B, T, Hq] natural-log LSE of the scaled logits, or NULL.
+ *   workspace   device scratch of at least rel_attn_workspace_bytes(shape,
+ *               num_splits) bytes, 256-byte aligned, prepared once with
+ *               rel_attn_workspace_init (it holds the device status word).
+ *
+ * Device-side problems (seq_len out of range, a block-table entry outside
+ * the pool, a wait that exceeded its bound) do not fault: they set bits in
+ * the workspace status word, read with rel_attn_read_status.  Rows of an
+ * offending sequence are written as NaN.
+ */
+int rel_attn_decode(const rel_attn_shape* shape, const void* q,
+                    const void* k_cache, const void* v_cache,
+                    const int32_t* block_table, const int32_t* seq_lens,
+                    const void* rel_table, int window, int num_splits,
+                    void* out, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * Split-phase form of rel_attn_decode, for callers that schedule the two
+ * kernels themselves (e.g. to time them apart, or to exchange per-split
+ * partials between devices before merging).  rel_attn_partial +
+ * rel_attn_combine with the same num_splits compute exactly what
+ * rel_attn_decode computes.  num_splits must be explicit here (1..256; use
+ * rel_attn_choose_splits).  With num_splits == 1 the partial call writes
+ * out/lse itself and the combine call is a no-op.  With num_splits > 1 the
+ * partial call writes the per-split (normalised output, lse) pairs into the
+ * workspace -- fp32 [S][B*T*Hq] lse after the 256-byte header, then fp32
+ * [S][B*T*Hq][D] outputs at the next 256-byte boundary; a split with no
+ * visible key holds lse = -inf and zeros -- and the combine call merges them:
+ *   lse = ln sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) o_s.
+ */
+int rel_attn_partial(const rel_attn_shape* shape, const void* q,
+                     const void* k_cache, const void* v_cache,
+                     const int32_t* block_table, const int32_t* seq_lens,
+                     const void* rel_table, int window, int num_splits,
+                     void* out, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
+                     float* lse, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* Bytes of workspace rel_attn_decode needs for this shape and split count
+ * (num_splits <= 0: the heuristic's choice).  0 when the shape is invalid. */
+size_t rel_attn_workspace_bytes(const rel_attn_shape* shape, int num_splits);
+
+/* Zero the workspace status word (asynchronous on `stream`).  Call once
+ * after allocating a workspace and after reading a non-zero status. */
+int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, read the workspace status word and clear it.
+ * Returns 0, REL_ATTN_ERR_TIMEOUT, REL_ATTN_ERR_BAD_SEQ or REL_ATTN_ERR_CUDA. */
+int rel_attn_read_status(void* workspace, void* stream);
+
+/* The split heuristic: KV splits per (sequence, KV head) so that
+ * batch * Hkv * splits fills `sm_count` SMs, bounded by the work available
+ * (at least one 128-key tile per split) and by 256.  sm_count <= 0 queries
+ * the current device.  Returns >= 1, or a negative error code. */
+int rel_attn_choose_splits(const rel_attn_shape* shape, int window, int sm_count);
+
+/* bucket(distance) exactly as the kernels compute it (host copy of the same
+ * edge table), for tests.  Returns -1 for an invalid shape or distance < 0. */
+int rel_attn_bucket(const rel_attn_shape* shape, int distance);
+
+/* Static description of an error code. */
+const char* rel_attn_error_string(int code);
+
+/* Library version, e.g. "rel_attn 0.1.0 sm_100a". */
+const char* rel_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REL_ATTN_H */

@@ -1,0 +1,455 @@
+// rel_attn.cu -- host side of the C ABI declared in include/rel_attn.h:
+// argument validation, the split heuristic, the bucket edge table, TMA
+// tensor-map encoding and the launches of the partial and combine kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "rel_attn.h"
+#include "rel_attn_kernels.cuh"
+
+namespace relattn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kHeaderBytes = 256;   // status word lives here
+
+struct DeviceInfo {
+  bool probed = false;
+  bool sm100 = false;
+  int sm_count = 0;
+  bool attr_set[4] = {false, false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool encode_fn_ready() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                         cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// Group width N (GQA group x query tokens, padded to the MMA N step of 16).
+int group_width(int G, int T) {
+  const int nq = G * T;
+  if (nq <= 16) return 16;
+  if (nq <= 32) return 32;
+  if (nq <= 48) return 48;
+  return 0;
+}
+
+int validate_shape(const rel_attn_shape* s) {
+  if (!s) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->batch > 65535) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->q_tokens < 1 || s->q_tokens > 8) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_kv_heads < 1 || s->num_kv_heads > 65535) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_q_heads < 1 || s->num_q_heads % s->num_kv_heads) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_q_heads / s->num_kv_heads != 6) return REL_ATTN_ERR_INVALID_ARG;
+  if (group_width(6, s->q_tokens) == 0) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->head_dim != kHeadDim || s->page_size != kPage) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_pages < 1 || s->max_pages_per_seq < 1) return REL_ATTN_ERR_INVALID_ARG;
+  if ((long long)s->num_pages * s->num_kv_heads * kPage >= (1ll << 31)) return REL_ATTN_ERR_INVALID_ARG;
+  if ((long long)s->max_pages_per_seq * kPage >= (1ll << 31)) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_buckets < 1 || s->exact_buckets < 1) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->num_buckets > s->exact_buckets) {
+    if (s->num_buckets - s->exact_buckets > kMaxTailBuckets) return REL_ATTN_ERR_INVALID_ARG;
+    if (s->max_distance <= s->exact_buckets) return REL_ATTN_ERR_INVALID_ARG;
+  }
+  if (s->max_seq_len < 0) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->out_fp32 != 0 && s->out_fp32 != 1) return REL_ATTN_ERR_INVALID_ARG;
+  return REL_ATTN_OK;
+}
+
+// Lower edges of the tail buckets.  e_k = ceil(E * (Dmax/E)^(k/NL)) in long
+// double; a value within 1e-9 (relative) of an integer is taken as that
+// integer so that exact powers (e.g. 1024 * 2^5) do not round up.
+void bucket_table(const rel_attn_shape* s, int* ex, int* nl, int* edges) {
+  const int NB = s->num_buckets, E = s->exact_buckets;
+  if (NB <= E) {
+    *ex = NB - 1;
+    *nl = 1;
+    edges[0] = NB - 1;
+    return;
+  }
+  const int n = NB - E;
+  *ex = E;
+  *nl = n;
+  const long double lr = log2l((long double)s->max_distance / (long double)E);
+  for (int k = 0; k <= n; ++k) {
+    const long double x = (long double)E * exp2l(lr * (long double)k / (long double)n);
+    const long double r = nearbyintl(x);
+    const long double e = (fabsl(x - r) <= 1e-9L * x) ? r : ceill(x);
+    edges[k] = (int)e;
+  }
+}
+
+// Small caches: the edge table depends only on (NB, E, Dmax) and a tensor
+// map only on (base pointer, extents); both are rebuilt otherwise per call.
+struct EdgeEntry { int nb = -1, e = -1, dmax = -1, ex = 0, nl = 0; int edges[kMaxTailBuckets + 1]; };
+struct MapEntry { const void* base = nullptr; uint64_t a = 0, b = 0; int kind = -1; CUtensorMap map; };
+constexpr int kEdgeCache = 4, kMapCache = 16;
+EdgeEntry g_edge_cache[kEdgeCache];
+MapEntry g_map_cache[kMapCache];
+int g_edge_next = 0, g_map_next = 0;
+std::mutex g_cache_mu;
+
+void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges) {
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  for (auto& e : g_edge_cache) {
+    if (e.nb == s->num_buckets && e.e == s->exact_buckets && e.dmax == s->max_distance) {
+      *ex = e.ex;
+      *nl = e.nl;
+      memcpy(edges, e.edges, sizeof(int) * (e.nl + 1));
+      return;
+    }
+  }
+  EdgeEntry& e = g_edge_cache[g_edge_next++ % kEdgeCache];
+  bucket_table(s, &e.ex, &e.nl, e.edges);
+  e.nb = s->num_buckets; e.e = s->exact_buckets; e.dmax = s->max_distance;
+  *ex = e.ex;
+  *nl = e.nl;
+  memcpy(edges, e.edges, sizeof(int) * (e.nl + 1));
+}
+
+int bucket_host(int d, int ex, int nl, const int* edges) {
+  if (d < ex) return d;
+  int lo = 0, hi = nl - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (edges[mid] <= d) lo = mid; else hi = mid - 1;
+  }
+  return ex + lo;
+}
+
+int splits_heuristic(const rel_attn_shape* s, int window, int sm_count) {
+  const long long cap = (long long)s->max_pages_per_seq * kPage;
+  long long max_len = (s->max_seq_len > 0) ? std::min<long long>(s->max_seq_len, cap) : cap;
+  long long visible = (window > 0) ? std::min<long long>(max_len, (long long)window + s->q_tokens - 1)
+                                   : max_len;
+  // a window may straddle one more page than it has keys for, but never more
+  // pages than the whole context: full attention bounds every window
+  const long long pages = std::min<long long>((visible + kPage - 1) / kPage + (window > 0 ? 1 : 0),
+                                              (max_len + kPage - 1) / kPage);
+  const long long tiles = (pages + 1) / 2;
+  const long long units = (long long)s->batch * s->num_kv_heads;
+  long long S;
+  if (units >= sm_count) S = (3LL * sm_count + units - 1) / units;   // several waves
+  else S = sm_count / units;                                          // one full wave
+  S = std::max<long long>(1, std::min<long long>(S, std::min<long long>(tiles, 256)));
+  return (int)S;
+}
+
+size_t workspace_for(const rel_attn_shape* s, int S) {
+  if (S <= 1) return kHeaderBytes;
+  const size_t rows = (size_t)s->batch * s->q_tokens * s->num_q_heads;
+  return kHeaderBytes + align256((size_t)S * rows * sizeof(float)) +
+         (size_t)S * rows * kHeadDim * sizeof(float);
+}
+
+int probe_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return REL_ATTN_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return REL_ATTN_ERR_NO_DEVICE;
+    }
+    di.sm100 = (prop.major == 10 && prop.minor == 0);
+    di.sm_count = prop.multiProcessorCount;
+    di.probed = true;
+  }
+  *dev_out = dev;
+  return di.sm100 ? REL_ATTN_OK : REL_ATTN_ERR_NO_DEVICE;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kPage};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_rel(CUtensorMap* m, const void* base, int NB, int Hkv) {
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)NB, (cuuint64_t)Hkv};
+  cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)NB * kHeadDim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kRChunkRows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64_t b) {
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    for (auto& e : g_map_cache)
+      if (e.kind == kind && e.base == base && e.a == a && e.b == b) { *out = e.map; return true; }
+  }
+  CUtensorMap m;
+  const bool ok = (kind == 2) ? make_map_rel(&m, base, (int)a, (int)b) : make_map_2d(&m, base, a);
+  if (!ok) return false;
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  MapEntry& e = g_map_cache[g_map_next++ % kMapCache];
+  e.kind = kind; e.base = base; e.a = a; e.b = b; e.map = m;
+  *out = m;
+  return true;
+}
+
+template <int N>
+int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di,
+                   int slot) {
+  auto kern = rel_attn_partial_kernel<N, 6>;
+  constexpr int smem = SmemLayout<N>::kAllocBytes;
+  if (!di.attr_set[slot]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return REL_ATTN_ERR_CUDA;
+    di.attr_set[slot] = true;
+  }
+  dim3 grid(S, Hkv, B);
+  kern<<<grid, kThreads, smem, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace relattn
+
+using namespace relattn;
+
+extern "C" {
+
+const char* rel_attn_version(void) { return "rel_attn 0.1.0 sm_100a"; }
+
+const char* rel_attn_error_string(int code) {
+  switch (code) {
+    case REL_ATTN_OK: return "success";
+    case REL_ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case REL_ATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case REL_ATTN_ERR_CUDA: return "CUDA runtime or launch failure";
+    case REL_ATTN_ERR_TIMEOUT: return "device-side bounded wait expired";
+    case REL_ATTN_ERR_BAD_SEQ: return "sequence length or block-table entry out of range";
+    case REL_ATTN_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown error";
+  }
+}
+
+size_t rel_attn_workspace_bytes(const rel_attn_shape* shape, int num_splits) {
+  if (validate_shape(shape) != REL_ATTN_OK || num_splits > 256) return 0;
+  int S = num_splits;
+  if (S <= 0) {
+    int dev;
+    const int sms = (probe_device(&dev) == REL_ATTN_OK) ? g_dev[dev].sm_count : 148;
+    S = splits_heuristic(shape, 0, sms);   // full attention bounds every window
+  }
+  return workspace_for(shape, S);
+}
+
+int rel_attn_choose_splits(const rel_attn_shape* shape, int window, int sm_count) {
+  const int rc = validate_shape(shape);
+  if (rc != REL_ATTN_OK) return rc;
+  if (sm_count <= 0) {
+    int dev;
+    const int prc = probe_device(&dev);
+    if (prc != REL_ATTN_OK) return prc;
+    sm_count = g_dev[dev].sm_count;
+  }
+  return splits_heuristic(shape, window, sm_count);
+}
+
+int rel_attn_bucket(const rel_attn_shape* shape, int distance) {
+  if (validate_shape(shape) != REL_ATTN_OK || distance < 0) return -1;
+  int ex, nl;
+  static thread_local int edges[kMaxTailBuckets + 1];
+  bucket_table_cached(shape, &ex, &nl, edges);
+  return bucket_host(distance, ex, nl, edges);
+}
+
+int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < kHeaderBytes) return REL_ATTN_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, kHeaderBytes, (cudaStream_t)stream) == cudaSuccess
+             ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
+}
+
+int rel_attn_read_status(void* workspace, void* stream) {
+  if (!workspace) return REL_ATTN_ERR_INVALID_ARG;
+  unsigned st = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return REL_ATTN_ERR_CUDA;
+  if (st == 0) return REL_ATTN_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(st), s) != cudaSuccess) return REL_ATTN_ERR_CUDA;
+  if (st & kStatusTimeout) return REL_ATTN_ERR_TIMEOUT;
+  return REL_ATTN_ERR_BAD_SEQ;
+}
+
+namespace {
+
+// Validation and parameter set-up shared by the entry points.  Returns the
+// resolved split count through *S.
+int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+            const int32_t* block_table, const int32_t* seq_lens, const void* rel_table, int window,
+            int num_splits, void* out, float* lse, void* workspace, size_t workspace_bytes,
+            DecodeParams* prm, int* S_out, DeviceInfo** di_out) {
+  // ---- validation (no CUDA call before this block passes)
+  int rc = validate_shape(shape);
+  if (rc != REL_ATTN_OK) return rc;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !rel_table || !out || !workspace)
+    return REL_ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+  if (misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) ||
+      misaligned(rel_table, 16) || misaligned(out, 16) || misaligned(workspace, 256) ||
+      misaligned(block_table, 4) || misaligned(seq_lens, 4) || (lse && misaligned(lse, 4)))
+    return REL_ATTN_ERR_INVALID_ARG;
+  if (num_splits > 256) return REL_ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < kHeaderBytes) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
+
+  int dev;
+  rc = probe_device(&dev);
+  if (rc != REL_ATTN_OK) return rc;
+  DeviceInfo& di = g_dev[dev];
+  const int S = (num_splits > 0) ? num_splits : splits_heuristic(shape, window, di.sm_count);
+  if (workspace_bytes < workspace_for(shape, S)) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  if (!encode_fn_ready()) return REL_ATTN_ERR_CUDA;
+
+  const int B = shape->batch, T = shape->q_tokens, Hq = shape->num_q_heads, Hkv = shape->num_kv_heads;
+  const size_t rows = (size_t)B * T * Hq;
+  memset(prm, 0, sizeof(*prm));
+  const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
+  if (!cached_map(&prm->tmap_k, 0, k_cache, kv_rows, 0) ||
+      !cached_map(&prm->tmap_v, 1, v_cache, kv_rows, 0) ||
+      !cached_map(&prm->tmap_r, 2, rel_table, (uint64_t)shape->num_buckets, (uint64_t)Hkv))
+    return REL_ATTN_ERR_CUDA;
+  prm->q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm->block_table = block_table;
+  prm->seq_lens = seq_lens;
+  prm->out = out;
+  prm->lse = lse;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  prm->status = reinterpret_cast<unsigned*>(ws);
+  prm->ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes);
+  prm->ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
+  prm->timeout_ns = kDefaultTimeoutNs;
+  prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
+  prm->num_pages = shape->num_pages;
+  prm->max_pages = shape->max_pages_per_seq;
+  prm->num_splits = S;
+  prm->window = window;
+  prm->out_fp32 = shape->out_fp32;
+  bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges);
+  prm->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
+  *S_out = S;
+  *di_out = &di;
+  return REL_ATTN_OK;
+}
+
+int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
+                       DeviceInfo& di) {
+  switch (group_width(6, shape->q_tokens)) {
+    case 16: return launch_partial<16>(prm, S, shape->batch, shape->num_kv_heads, st, di, 0);
+    case 32: return launch_partial<32>(prm, S, shape->batch, shape->num_kv_heads, st, di, 1);
+    case 48: return launch_partial<48>(prm, S, shape->batch, shape->num_kv_heads, st, di, 2);
+    default: return REL_ATTN_ERR_INVALID_ARG;
+  }
+}
+
+// LSE-merge launch; programmatic dependent launch lets it start while the
+// partial kernel drains (it waits on griddepcontrol before reading).
+int launch_combine(const rel_attn_shape* shape, int S, void* out, float* lse, void* workspace,
+                   cudaStream_t st) {
+  const size_t rows = (size_t)shape->batch * shape->q_tokens * shape->num_q_heads;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  const float* ws_lse = reinterpret_cast<const float*>(ws + kHeaderBytes);
+  const float* ws_o = reinterpret_cast<const float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, rel_attn_combine_kernel, ws_lse, ws_o, S, (int)rows, out, lse,
+                         shape->out_fp32) != cudaSuccess) {
+    cudaGetLastError();
+    return REL_ATTN_ERR_CUDA;
+  }
+  return REL_ATTN_OK;
+}
+
+}  // namespace
+
+int rel_attn_decode(const rel_attn_shape* shape, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_table, const int32_t* seq_lens,
+                    const void* rel_table, int window, int num_splits, void* out, float* lse,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeParams prm;
+  int S = 0;
+  DeviceInfo* di = nullptr;
+  int rc = prepare(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, num_splits,
+                   out, lse, workspace, workspace_bytes, &prm, &S, &di);
+  if (rc != REL_ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = launch_partial_any(prm, shape, S, st, *di);
+  if (rc != REL_ATTN_OK || S == 1) return rc;
+  return launch_combine(shape, S, out, lse, workspace, st);
+}
+
+int rel_attn_partial(const rel_attn_shape* shape, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_table, const int32_t* seq_lens,
+                     const void* rel_table, int window, int num_splits, void* out, float* lse,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (num_splits < 1) return REL_ATTN_ERR_INVALID_ARG;
+  DecodeParams prm;
+  int S = 0;
+  DeviceInfo* di = nullptr;
+  int rc = prepare(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, num_splits,
+                   out, lse, workspace, workspace_bytes, &prm, &S, &di);
+  if (rc != REL_ATTN_OK) return rc;
+  return launch_partial_any(prm, shape, S, reinterpret_cast<cudaStream_t>(stream), *di);
+}
+
+int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, float* lse,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_shape(shape);
+  if (rc != REL_ATTN_OK) return rc;
+  if (num_splits < 1 || num_splits > 256 || !out || !workspace) return REL_ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return REL_ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < workspace_for(shape, num_splits)) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  if (num_splits == 1) return REL_ATTN_OK;
+  int dev;
+  rc = probe_device(&dev);
+  if (rc != REL_ATTN_OK) return rc;
+  return launch_combine(shape, num_splits, out, lse, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

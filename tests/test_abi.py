@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the header declares, validates arguments before touching CUDA, and its host
+copy of the bucket table (the one handed to the kernels) equals the oracle's
+bucket function bit for bit."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from relative_bias_gqa_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ra():
+    build_mod.build()
+    from relative_bias_gqa_b200 import rel_attn
+    return rel_attn
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "rel_attn.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(rel_attn_\w+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(ra):
+    names = header_functions()
+    assert set(names) == set(ra.EXPORTED)
+    lib = ctypes.CDLL(build_mod.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert "sm_100a" in ra.version()
+
+
+def shape(ra, **kw):
+    base = dict(batch=1, q_tokens=1, num_q_heads=48, num_kv_heads=8, num_pages=1563,
+                max_pages_per_seq=1563, num_buckets=1280, max_seq_len=100_000)
+    base.update(kw)
+    return ra.make_shape(**base)
+
+
+@pytest.mark.parametrize("nb", [1280, 1024, 1030, 8, 1])
+def test_host_bucket_table_matches_oracle(ra, nb):
+    import oracle
+    s = shape(ra, num_buckets=nb)
+    d = np.concatenate([np.arange(0, 70_000), np.arange(70_000, 1 << 21, 7),
+                        [(1 << 20) - 1, 1 << 20, (1 << 20) + 1, 5 << 20]])
+    want = oracle.bucket_of_distance(d, nb)
+    f = ra.lib.rel_attn_bucket
+    got = np.array([f(ctypes.byref(s), int(x)) for x in d])
+    assert np.array_equal(got, want)
+    assert f(ctypes.byref(s), -1) == -1
+
+
+def test_host_bucket_every_distance_nb1280(ra):
+    import oracle
+    s = shape(ra)
+    e = oracle.log_bucket_edges(1280)
+    # every edge and its neighbours
+    d = np.unique(np.concatenate([e - 1, e, e + 1]))
+    d = d[d >= 0]
+    got = np.array([ra.rel_attn_bucket(s, int(x)) for x in d])
+    assert np.array_equal(got, oracle.bucket_of_distance(d, 1280))
+
+
+BAD = [
+    dict(q_tokens=0), dict(q_tokens=9), dict(head_dim=64), dict(page_size=16),
+    dict(num_q_heads=47), dict(num_q_heads=64), dict(num_kv_heads=0), dict(batch=0),
+    dict(num_buckets=0), dict(num_buckets=1024 + 513), dict(num_pages=0),
+    dict(max_pages_per_seq=0), dict(out_fp32=2), dict(max_seq_len=-1),
+    dict(num_pages=1 << 23),
+]
+
+
+@pytest.mark.parametrize("kw", BAD)
+def test_invalid_shape_rejected_before_any_cuda_call(ra, kw):
+    s = shape(ra, **kw)
+    fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+    rc = ra.lib.rel_attn_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 0, 0,
+                                fake, None, fake, 1 << 30, None)
+    assert rc == ra.REL_ATTN_ERR_INVALID_ARG
+    assert ra.rel_attn_workspace_bytes(s, 4) == 0
+
+
+def test_invalid_pointers_and_splits(ra):
+    s = shape(ra)
+    f = ctypes.c_void_p(1 << 20)
+    call = ra.lib.rel_attn_decode
+    assert call(ctypes.byref(s), None, f, f, f, f, f, 0, 0, f, None, f, 1 << 30, None) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert call(ctypes.byref(s), f, f, f, f, f, f, 0, 257, f, None, f, 1 << 30, None) == ra.REL_ATTN_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert call(ctypes.byref(s), odd, f, f, f, f, f, 0, 0, f, None, f, 1 << 30, None) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert call(ctypes.byref(s), f, f, f, f, f, f, 0, 0, f, None, odd, 1 << 30, None) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert call(ctypes.byref(s), f, f, f, f, f, f, 0, 0, f, None, f, 16, None) == ra.REL_ATTN_ERR_WORKSPACE_TOO_SMALL
+    assert call(None, f, f, f, f, f, f, 0, 0, f, None, f, 1 << 30, None) == ra.REL_ATTN_ERR_INVALID_ARG
+
+
+def test_split_heuristic_values(ra):
+    # 148 SMs: batch-1 48/8 fills one wave with 18 splits per KV head
+    assert ra.rel_attn_choose_splits(shape(ra), 0, 148) == 18
+    # a sliding window of 1,024 has 9 tiles: never more splits than tiles
+    assert ra.rel_attn_choose_splits(shape(ra), 1024, 148) == 9
+    # small contexts: at most one split per 128-key tile
+    assert ra.rel_attn_choose_splits(shape(ra, max_seq_len=300), 0, 148) == 3
+    # 32 sequences x 8 heads > 148 SMs: a few splits for load balance
+    s = shape(ra, batch=32, max_seq_len=131_072, max_pages_per_seq=2048, num_pages=40000)
+    v = ra.rel_attn_choose_splits(s, 0, 148)
+    assert 1 <= v <= 4
+    for sm in (1, 7, 148, 1000):
+        assert 1 <= ra.rel_attn_choose_splits(shape(ra), 0, sm) <= 256
+
+
+def test_workspace_bytes(ra):
+    s = shape(ra)
+    assert ra.rel_attn_workspace_bytes(s, 1) == 256
+    rows = 48
+    want = 256 + ((18 * rows * 4 + 255) // 256) * 256 + 18 * rows * 128 * 4
+    assert ra.rel_attn_workspace_bytes(s, 18) == want
+    assert ra.rel_attn_workspace_bytes(s, 256) > ra.rel_attn_workspace_bytes(s, 18)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_no_device_reported_without_gpu(ra):
+    s = shape(ra)
+    f = ctypes.c_void_p(1 << 20)
+    rc = ra.lib.rel_attn_decode(ctypes.byref(s), f, f, f, f, f, f, 0, 4, f, None, f, 1 << 30, None)
+    assert rc == ra.REL_ATTN_ERR_NO_DEVICE
+
+
+def test_error_strings(ra):
+    for code in range(-6, 1):
+        assert ra.error_string(code) and ra.error_string(code) != "unknown error"
