@@ -129,6 +129,38 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
                      float* lse, void* workspace, size_t workspace_bytes,
                      void* stream);
 
+/*
+ * rel_attn_decode_static -- rel_attn_decode without a workspace argument.
+ * (An addition of this library; the pages describe nothing like it.)
+ *
+ * For callers that cannot allocate device memory: for example a plugin that a
+ * host framework hands only its input and output buffers, or a serving engine
+ * that has reserved all of HBM for its KV cache so that another cudaMalloc
+ * would fail.  The scratch space comes from a fixed array inside the library
+ * (REL_ATTN_STATIC_SCRATCH_BYTES = 4 MiB, held on every GPU that loads the
+ * library until the process exits); this entry point itself allocates nothing.
+ *
+ *   - Arguments are those of rel_attn_decode minus the workspace.
+ *   - Shapes whose workspace (rel_attn_workspace_bytes(shape, num_splits))
+ *     exceeds 4 MiB are rejected with REL_ATTN_ERR_WORKSPACE_TOO_SMALL before
+ *     anything is launched; pass a smaller num_splits or use rel_attn_decode.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents (each call clears the status word it needs).  Calls that
+ *     overlap on the GPU -- on different streams, or from different host
+ *     threads -- race on it; serialise them.
+ *   - Device-side status is not reported (there is no workspace to read it
+ *     from): rejected sequences still come back as NaN rows.
+ */
+#define REL_ATTN_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+int rel_attn_decode_static(const rel_attn_shape* shape, const void* q,
+                           const void* k_cache, const void* v_cache,
+                           const int32_t* block_table, const int32_t* seq_lens,
+                           const void* rel_table, int window, int num_splits,
+                           void* out, float* lse, void* stream);
+
 /* Bytes of workspace rel_attn_decode needs for this shape and split count
  * (num_splits <= 0: the heuristic's choice).  0 when the shape is invalid. */
 size_t rel_attn_workspace_bytes(const rel_attn_shape* shape, int num_splits);

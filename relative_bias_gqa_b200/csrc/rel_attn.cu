@@ -453,3 +453,82 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, flo
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.
+//
+// Some callers have no way to allocate device memory: a plugin that is handed
+// only its input and output buffers by a host framework, or a serving engine
+// that reserves all of HBM for its KV cache up front, so that an extra
+// cudaMalloc fails.  rel_attn_decode_static lets them run the operation with
+// the scratch space (device status word + per-split partial results) taken
+// from a fixed array compiled into this library instead of a caller-owned
+// workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;   // 4 MiB on every device
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+void* g_static_scratch_addr[kMaxDevices];
+std::mutex g_static_mu;
+
+// Device address of the array on the current device, looked up once per
+// device.  In host code the array's name is only a host-side stand-in, so the
+// kernels must be given this address, never the symbol itself.
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return REL_ATTN_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return REL_ATTN_ERR_CUDA;
+    }
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return REL_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int rel_attn_decode_static(const rel_attn_shape* shape, const void* q,
+                                      const void* k_cache, const void* v_cache,
+                                      const int32_t* block_table, const int32_t* seq_lens,
+                                      const void* rel_table, int window, int num_splits,
+                                      void* out, float* lse, void* stream) {
+  int rc = validate_shape(shape);
+  if (rc != REL_ATTN_OK) return rc;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !rel_table || !out)
+    return REL_ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+  if (misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) ||
+      misaligned(rel_table, 16) || misaligned(out, 16) || misaligned(block_table, 4) ||
+      misaligned(seq_lens, 4) || (lse && misaligned(lse, 4)))
+    return REL_ATTN_ERR_INVALID_ARG;
+  if (num_splits > 256) return REL_ATTN_ERR_INVALID_ARG;
+  int dev;
+  rc = probe_device(&dev);
+  if (rc != REL_ATTN_OK) return rc;
+  const int S = (num_splits > 0) ? num_splits : splits_heuristic(shape, window, g_dev[dev].sm_count);
+  if (workspace_for(shape, S) > kStaticScratchBytes) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  rc = static_scratch_address(&scratch);
+  if (rc != REL_ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps whatever the previous call left there: the status word
+  // must start at zero; the per-split partials are rewritten in full.
+  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, st) != cudaSuccess) {
+    cudaGetLastError();
+    return REL_ATTN_ERR_CUDA;
+  }
+  return rel_attn_decode(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, S,
+                         out, lse, scratch, kStaticScratchBytes, stream);
+}

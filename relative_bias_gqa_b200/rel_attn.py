@@ -26,7 +26,7 @@ REL_ATTN_ERR_NO_DEVICE = -6
 EXPORTED = (
     "rel_attn_decode", "rel_attn_partial", "rel_attn_combine", "rel_attn_workspace_bytes", "rel_attn_workspace_init",
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
-    "rel_attn_error_string", "rel_attn_version",
+    "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
 )
 
 
@@ -56,6 +56,9 @@ def _load():
     lib.rel_attn_partial.restype = ctypes.c_int
     lib.rel_attn_combine.argtypes = [SP, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
     lib.rel_attn_combine.restype = ctypes.c_int
+    lib.rel_attn_decode_static.argtypes = [SP, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                           P, P, P]
+    lib.rel_attn_decode_static.restype = ctypes.c_int
     lib.rel_attn_workspace_bytes.argtypes = [SP, ctypes.c_int]
     lib.rel_attn_workspace_bytes.restype = ctypes.c_size_t
     lib.rel_attn_workspace_init.argtypes = [P, ctypes.c_size_t, P]
