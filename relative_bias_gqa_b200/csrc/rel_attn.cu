@@ -46,9 +46,10 @@ bool encode_fn_ready() {
 }
 
 // Group width N (GQA group x query tokens, padded to the MMA N step of 16).
+// The 16-wide instance (two softmax groups) serves up to 6 live rows.
 int group_width(int G, int T) {
   const int nq = G * T;
-  if (nq <= 16) return 16;
+  if (nq <= 6) return 16;
   if (nq <= 32) return 32;
   if (nq <= 48) return 48;
   return 0;
@@ -194,10 +195,10 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows) {
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_map_rel(CUtensorMap* m, const void* base, int NB, int Hkv) {
+bool make_map_rel(CUtensorMap* m, const void* base, int NB, int Hkv, int box_rows) {
   cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)NB, (cuuint64_t)Hkv};
   cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)NB * kHeadDim * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kRChunkRows, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -211,7 +212,9 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
       if (e.kind == kind && e.base == base && e.a == a && e.b == b) { *out = e.map; return true; }
   }
   CUtensorMap m;
-  const bool ok = (kind == 2) ? make_map_rel(&m, base, (int)a, (int)b) : make_map_2d(&m, base, a);
+  // kinds: 0 = K pool, 1 = V pool, 2 / 3 = relative table with 136- / 128-row boxes
+  const bool ok = (kind >= 2) ? make_map_rel(&m, base, (int)a, (int)b, kind == 2 ? 136 : 128)
+                              : make_map_2d(&m, base, a);
   if (!ok) return false;
   std::lock_guard<std::mutex> lk(g_cache_mu);
   MapEntry& e = g_map_cache[g_map_next++ % kMapCache];
@@ -220,18 +223,19 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
   return true;
 }
 
-template <int N>
+template <int N, int NG>
 int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di,
                    int slot) {
-  auto kern = rel_attn_partial_kernel<N, 6>;
-  constexpr int smem = SmemLayout<N>::kAllocBytes;
+  using KC = KernelConfig<N, NG>;
+  auto kern = rel_attn_partial_kernel<N, 6, NG>;
+  constexpr int smem = KC::kAllocBytes;
   if (!di.attr_set[slot]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return REL_ATTN_ERR_CUDA;
     di.attr_set[slot] = true;
   }
   dim3 grid(S, Hkv, B);
-  kern<<<grid, kThreads, smem, st>>>(prm);
+  kern<<<grid, KC::kThreads, smem, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
 }
 
@@ -342,7 +346,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
   if (!cached_map(&prm->tmap_k, 0, k_cache, kv_rows, 0) ||
       !cached_map(&prm->tmap_v, 1, v_cache, kv_rows, 0) ||
-      !cached_map(&prm->tmap_r, 2, rel_table, (uint64_t)shape->num_buckets, (uint64_t)Hkv))
+      !cached_map(&prm->tmap_r, group_width(6, T) == 16 ? 3 : 2, rel_table,
+                  (uint64_t)shape->num_buckets, (uint64_t)Hkv))
     return REL_ATTN_ERR_CUDA;
   prm->q = reinterpret_cast<const __nv_bfloat16*>(q);
   prm->block_table = block_table;
@@ -370,9 +375,9 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
 int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
                        DeviceInfo& di) {
   switch (group_width(6, shape->q_tokens)) {
-    case 16: return launch_partial<16>(prm, S, shape->batch, shape->num_kv_heads, st, di, 0);
-    case 32: return launch_partial<32>(prm, S, shape->batch, shape->num_kv_heads, st, di, 1);
-    case 48: return launch_partial<48>(prm, S, shape->batch, shape->num_kv_heads, st, di, 2);
+    case 16: return launch_partial<16, 2>(prm, S, shape->batch, shape->num_kv_heads, st, di, 0);
+    case 32: return launch_partial<32, 1>(prm, S, shape->batch, shape->num_kv_heads, st, di, 1);
+    case 48: return launch_partial<48, 1>(prm, S, shape->batch, shape->num_kv_heads, st, di, 2);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }

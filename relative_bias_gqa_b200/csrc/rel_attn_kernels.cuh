@@ -11,11 +11,16 @@
 //                 S^T = K . Q^T           (128 keys x N)
 //                 X^T = R_chunk . Q^T     (136 relative rows x N)
 //                 O^T = V^T . P^T         (128 dims x N)
-//   warps 2-5   softmax (128 threads, one key / one head-dim lane each):
-//               tcgen05.ld of S^T, relative term sheared into place through a
-//               shared-memory table indexed by bucket(distance), masks,
-//               fp32 online softmax in the log2 domain, P to shared memory
-//               (bf16, 128B-swizzled), O^T tiles accumulated in registers.
+//   softmax     NG groups of 4 warps (one key / one head-dim lane per thread);
+//               with two groups, group g takes the tiles i with i % 2 == g, so
+//               two tiles' softmax run at once (each group keeps its own
+//               running max / sum / output and its own relative-row chunk;
+//               the two partial states are merged by LSE at the end).  Per
+//               tile: tcgen05.ld of S^T, relative term sheared into place
+//               through a shared-memory table indexed by bucket(distance),
+//               masks, fp32 online softmax in the log2 domain, P to shared
+//               memory (bf16 hi + lo, 128B-swizzled), O^T tile accumulated in
+//               registers.
 // Combine kernel: LSE-merge of the per-split partial results.
 //
 // The dense relative product followed by a distance-indexed gather is the
@@ -43,17 +48,17 @@ namespace relattn {
 constexpr int kHeadDim = 128;
 constexpr int kPage = 64;
 constexpr int kTileKeys = 128;                 // two pages per tile
-constexpr int kRChunkRows = 136;               // relative-table rows per chunk
 constexpr int kMaxTailBuckets = 512;           // log buckets supported
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kStageBytes = 65536;             // K (32 KB) + V (32 KB)
+constexpr int kSoftmaxThreads = 128;           // one softmax group
+constexpr int kVSlotBytes = 32768;             // V tile: 128 keys x 128 dims bf16
 constexpr int kHalfTileBytes = 16384;          // 128 rows x 128 B (one 64-dim half)
 constexpr int kPageHalfBytes = 8192;           // 64 rows x 128 B
-constexpr int kRHalfBytes = kRChunkRows * 128; // 17408
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadSeq = 2u;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s
+// Lazy-max slack (log2 units): p = exp2(x - m_ref) may reach 2^64, far
+// inside fp32 / bf16 range even summed over 2^31 keys.
+constexpr float kLazyLog2 = 64.f;
 
 struct alignas(64) DecodeParams {
   CUtensorMap tmap_k;   // K pool viewed as [num_pages*Hkv*P rows, 128] bf16
@@ -77,30 +82,53 @@ struct alignas(64) DecodeParams {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// Shared-memory carve-up for an N-wide (padded group) tile.
-template <int N>
-struct SmemLayout {
-  static constexpr int kStages = (N == 16) ? 3 : 2;
-  static constexpr int kYStride = N + 1;                       // odd: conflict-free gathers
+// Compile-time configuration of one kernel instance: N = padded group width
+// (G heads x T tokens rounded up to the MMA N step), NG = softmax groups.
+// K tiles and relative-row chunks share one ring of slots (each slot is
+// released as soon as its MMA has read it); V tiles have their own, deeper
+// ring (a V slot is held until the P.V product of its tile).
+template <int N, int NG>
+struct KernelConfig {
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
+  // relative rows per chunk: 128 cover one 128-key tile for one token; with
+  // T tokens a tile needs 127 + T rows
+  static constexpr int kRows = (N == 16) ? 128 : 136;
+  static constexpr int kRHalfBytes = kRows * 128;
+  static constexpr int kKSlotBytes = 2 * kRHalfBytes;          // >= one K tile (32 KB)
+  static constexpr int kKSlots = 2;
+  static constexpr int kVSlots = (N == 16) ? 4 : (N == 32 ? 3 : 2);
+  // Relative-table gather stride: odd for conflict-free gathers.  The N = 16
+  // instance serves at most 6 live rows.
+  static constexpr int kYStride = (N == 16) ? 7 : N + 1;
   static constexpr int kOperandBytes = 2 * N * 128;            // N rows x 128 dims, two 64-dim halves
-  static constexpr int oQ = kStages * kStageBytes;
-  static constexpr int oP = oQ + kOperandBytes;                // two P buffers, each hi + lo
-  static constexpr int kPBufBytes = 2 * kOperandBytes;
-  static constexpr int oY = oP + 2 * kPBufBytes;
-  static constexpr int oRed = oY + align_up(kRChunkRows * kYStride * 4, 16);
-  static constexpr int oLred = oRed + 2 * 4 * N * 4;
-  static constexpr int oAlpha = oLred + 4 * N * 4;
-  static constexpr int oM = oAlpha + 2 * N * 4;
-  static constexpr int oEdges = oM + 2 * N * 4;
+  static constexpr int kPBufBytes = 2 * kOperandBytes;         // [P_hi; P_lo]: 128 keys x 2N rows
+  static constexpr int kYBytes = align_up(kRows * kYStride * 4, 16);
+  static constexpr int oK = 0;
+  static constexpr int oV = kKSlots * kKSlotBytes;
+  static constexpr int oQ = oV + kVSlots * kVSlotBytes;
+  static constexpr int oP = oQ + kOperandBytes;                // two P buffers
+  static constexpr int oY = oP + 2 * kPBufBytes;               // one table per group
+  static constexpr int oRed = oY + NG * kYBytes;               // [NG][2][4][N]
+  static constexpr int oLred = oRed + NG * 2 * 4 * N * 4;      // [NG][4][N]
+  static constexpr int oAlpha = oLred + NG * 4 * N * 4;        // [NG][2][N]
+  static constexpr int oEdges = oAlpha + NG * 2 * N * 4;
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
-  // barriers: full[S], empty[S], s_full[2], s_empty[2], p_full[2], o_full[2],
-  //           o_empty[2], x_full, x_empty, drain
-  static constexpr int kNumBars = 2 * kStages + 13;
+  // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s_full[2],
+  //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[NG],
+  //           x_empty[NG], drain
+  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 11 + 2 * NG;
   static constexpr int oMisc = oBar + kNumBars * 8;            // tmem base, abort flag
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAllocBytes = kBytes + 1024;            // 1024-byte alignment slack
-  static constexpr int kTmemCols = (6 * N <= 128) ? 128 : (6 * N <= 256 ? 256 : 512);
+  // TMEM columns: S[2] (N each), O[2] (2N each: the P_hi and P_lo halves),
+  // per group X0 (and X1 for 136-row chunks)
+  static constexpr int kXCols = (kRows > 128) ? 2 * N : N;
+  static constexpr int kTmemUsed = 6 * N + kXCols * NG;
+  static constexpr int kTmemCols = (kTmemUsed <= 128) ? 128 : (kTmemUsed <= 256 ? 256 : 512);
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
+  static_assert(kKSlotBytes >= 2 * kHalfTileBytes && oV % 1024 == 0 && oQ % 1024 == 0,
+                "slot layout");
+  static_assert(oV >= N * 128 * 4 + 2 * N * 4, "exchange area");
 };
 
 // Per-CTA geometry shared by the three roles.
@@ -115,9 +143,10 @@ struct TilePlan {
   bool chunk;   // a new relative-row chunk must be loaded before this tile
 };
 
-// Cursor state carried from tile to tile.  Distances only shrink as the walk
-// moves to later keys, so the tail-bucket indices are found by stepping the
-// cursors down the edge table instead of searching it.
+// Cursor state carried from tile to tile (one per softmax group: a group's
+// tiles are planned against its own relative-row chunk).  Distances only
+// shrink as the walk moves to later keys, so the tail-bucket indices are found
+// by moving the cursors down the edge table.
 struct PlanState {
   int c0 = 0;
   bool have = false;
@@ -125,14 +154,26 @@ struct PlanState {
   __device__ explicit PlanState(int nl) : k_hi(nl - 1), k_lo(nl - 1) {}
 };
 
+// Largest k' <= k with edges[k'] <= d (edges[0] <= d is guaranteed): a few
+// linear steps, then a binary search for long moves.
 __device__ __forceinline__ int step_down(int k, int d, const int* edges) {
-  while (k > 0 && edges[k] > d) --k;
-  return k;
+#pragma unroll 1
+  for (int s = 0; s < 4; ++s) {
+    if (k == 0 || edges[k] <= d) return k;
+    --k;
+  }
+  int lo = 0, hi = k;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (edges[mid] <= d) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // Decides, for tile ti, the loaded pages and whether the relative-row chunk
-// [c0, c0+136) must move so that it covers every bucket the tile needs.
+// [c0, c0+ROWS) must move so that it covers every bucket the tile needs.
 // All roles call it with identical arguments, so they agree on the sequence.
+template <int ROWS>
 __device__ __forceinline__ TilePlan plan_tile(const SplitGeom& g, int ti, int ex, const int* edges,
                                               PlanState& st) {
   TilePlan t;
@@ -155,9 +196,9 @@ __device__ __forceinline__ TilePlan plan_tile(const SplitGeom& g, int ti, int ex
     st.k_lo = step_down(st.k_lo, d_lo, edges);
     b_lo = ex + st.k_lo;
   }
-  t.chunk = !(st.have && b_lo >= st.c0 && b_hi < st.c0 + kRChunkRows);
+  t.chunk = !(st.have && b_lo >= st.c0 && b_hi < st.c0 + ROWS);
   if (t.chunk) {
-    st.c0 = max(0, b_hi - (kRChunkRows - 1));
+    st.c0 = max(0, b_hi - (ROWS - 1));
     st.have = true;
   }
   return t;
@@ -195,12 +236,14 @@ __device__ void fill_rows(const DecodeParams& p, int b, int h, int s, float o_va
   }
 }
 
-template <int N, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int N, int G, int NG>
+__global__ void __launch_bounds__(KernelConfig<N, NG>::kThreads, 1)
 rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
-  using SL = SmemLayout<N>;
-  constexpr int STG = SL::kStages;
-  constexpr int YS = SL::kYStride;
+  using KC = KernelConfig<N, NG>;
+  constexpr int KS = KC::kKSlots;
+  constexpr int VS = KC::kVSlots;
+  constexpr int ROWS = KC::kRows;
+  constexpr int YS = KC::kYStride;
   constexpr int TMAX = (N + G - 1) / G;
 
   extern __shared__ uint8_t smem_raw[];
@@ -213,6 +256,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int T = p.T;
   const int NQ = T * G;
+  RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
@@ -241,36 +285,40 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   }
 
   // --------------------------------------------------------- smem carve-up
-  const uint32_t sQ = sbase + SL::oQ;
-  const uint32_t sP0 = sbase + SL::oP;
-  float* Y = reinterpret_cast<float*>(smem + SL::oY);
-  float* red = reinterpret_cast<float*>(smem + SL::oRed);
-  float* lred = reinterpret_cast<float*>(smem + SL::oLred);
-  float* alpha_buf = reinterpret_cast<float*>(smem + SL::oAlpha);
-  float* m_buf = reinterpret_cast<float*>(smem + SL::oM);
-  int* s_edges = reinterpret_cast<int*>(smem + SL::oEdges);
-  const uint32_t bar0 = sbase + SL::oBar;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STG + s); };
-  const uint32_t s_full = bar0 + 8u * (2 * STG + 0);    // +8*buf
-  const uint32_t s_empty = bar0 + 8u * (2 * STG + 2);
-  const uint32_t p_full = bar0 + 8u * (2 * STG + 4);
-  const uint32_t o_full = bar0 + 8u * (2 * STG + 6);
-  const uint32_t o_empty = bar0 + 8u * (2 * STG + 8);
-  const uint32_t x_full = bar0 + 8u * (2 * STG + 10);
-  const uint32_t x_empty = bar0 + 8u * (2 * STG + 11);
-  const uint32_t drain_bar = bar0 + 8u * (2 * STG + 12);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL::oMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::oMisc + 4);
-  auto stage_addr = [&](int k) { return sbase + (uint32_t)((k % STG) * kStageBytes); };
+  const uint32_t sQ = sbase + KC::oQ;
+  const uint32_t sP0 = sbase + KC::oP;
+  int* s_edges = reinterpret_cast<int*>(smem + KC::oEdges);
+  const uint32_t bar0 = sbase + KC::oBar;
+  // K ring (K tiles and relative-row chunks) and V ring, each a full/empty pair
+  auto kfull = [&](int s) { return bar0 + 8u * s; };
+  auto kempty = [&](int s) { return bar0 + 8u * (KS + s); };
+  auto vfull = [&](int s) { return bar0 + 8u * (2 * KS + s); };
+  auto vempty = [&](int s) { return bar0 + 8u * (2 * KS + VS + s); };
+  constexpr int kB = 2 * KS + 2 * VS;
+  const uint32_t s_full = bar0 + 8u * (kB + 0);    // +8*buf
+  const uint32_t s_empty = bar0 + 8u * (kB + 2);
+  const uint32_t p_full = bar0 + 8u * (kB + 4);
+  const uint32_t o_full = bar0 + 8u * (kB + 6);
+  const uint32_t o_empty = bar0 + 8u * (kB + 8);
+  const uint32_t x_full = bar0 + 8u * (kB + 10);   // +8*group
+  const uint32_t x_empty = bar0 + 8u * (kB + 10 + NG);
+  const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * NG);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 4);
+  auto kslot = [&](int k) { return sbase + KC::oK + (uint32_t)((k % KS) * KC::kKSlotBytes); };
+  auto vslot = [&](int i) { return sbase + KC::oV + (uint32_t)((i % VS) * kVSlotBytes); };
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
   if (warp == 0) {
     if (lane == 0) {
-      for (int s = 0; s < STG; ++s) {
-        ptx::mbar_init(full_bar(s), 1);
-        ptx::mbar_init(empty_bar(s), 1);
+      for (int s = 0; s < KS; ++s) {
+        ptx::mbar_init(kfull(s), 1);
+        ptx::mbar_init(kempty(s), 1);
+      }
+      for (int s = 0; s < VS; ++s) {
+        ptx::mbar_init(vfull(s), 1);
+        ptx::mbar_init(vempty(s), 1);
       }
       for (int i = 0; i < 2; ++i) {
         ptx::mbar_init(s_full + 8u * i, 1);
@@ -279,8 +327,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         ptx::mbar_init(o_full + 8u * i, 1);
         ptx::mbar_init(o_empty + 8u * i, kSoftmaxThreads);
       }
-      ptx::mbar_init(x_full, 1);
-      ptx::mbar_init(x_empty, kSoftmaxThreads);
+      for (int gq = 0; gq < NG; ++gq) {
+        ptx::mbar_init(x_full + 8u * gq, 1);
+        ptx::mbar_init(x_empty + 8u * gq, kSoftmaxThreads);
+      }
       ptx::mbar_init(drain_bar, 1);
       *abort_flag = 0;
       ptx::fence_mbar_init();
@@ -289,12 +339,13 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       ptx::prefetch_tmap(&p.tmap_r);
     }
   } else if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), SL::kTmemCols);
+    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), KC::kTmemCols);
     ptx::tmem_relinquish();
   } else {
     const int st = tid - 64;
+    const int nst = kSoftmaxThreads * NG;
     // Q group tile: rows n = t*G + g (padding rows zero), 128B-swizzled K-major.
-    for (int u = st; u < N * 16; u += kSoftmaxThreads) {
+    for (int u = st; u < N * 16; u += nst) {
       const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (n < NQ) {
@@ -303,17 +354,18 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
                                    + half * 64 + w16 * 8;
         v = __ldg(reinterpret_cast<const uint4*>(src));
       }
-      uint8_t* dst = smem + SL::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4);
+      uint8_t* dst = smem + KC::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4);
       *reinterpret_cast<uint4*>(dst) = v;
     }
-    for (int e = st; e <= p.nl; e += kSoftmaxThreads) s_edges[e] = p.edges[e];
-    for (int e = st; e < 2 * N; e += kSoftmaxThreads) m_buf[e] = -INFINITY;
+    for (int e = st; e <= p.nl; e += nst) s_edges[e] = p.edges[e];
     ptx::fence_proxy_async_smem();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const uint32_t tS = tmem, tO = tmem + 2 * N;                         // O buffer b at +2N*b
+  auto tX = [&](int gq) { return tmem + 6 * N + KC::kXCols * gq; };   // X0; X1 at +N
 
   // ------------------------------------------------------------- producer
   if (warp == 0) {
@@ -325,56 +377,76 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     };
     int bt_cur = bt_load(0);
     int bt_next = bt_load(1);
-    int k = 0;
-    PlanState ps(p.nl);
+    int k = 0;                                // K-ring items issued
+    int i_v = 0;                              // V-ring items (= tiles) issued
+    PlanState ps0(p.nl), ps1(p.nl);
     bool ok = true, bad_page = false;
     for (int ti = 0; ti < g.ntiles; ++ti) {
       if (ti > 0 && (ti & 15) == 0) {
         bt_cur = bt_next;
         bt_next = bt_load((ti >> 4) + 1);
       }
-      const TilePlan tp = plan_tile(g, ti, p.ex, s_edges, ps);
+      const bool odd = (NG == 2) && (ti & 1);
+      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, odd ? ps1 : ps0);
+      const int c0 = odd ? ps1.c0 : ps0.c0;
       if (tp.chunk) {
         ok = __all_sync(0xffffffffu,
-                        ptx::mbar_wait(empty_bar(k % STG), ((k / STG) & 1) ^ 1, abort_flag, tlim));
+                        ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
         if (!ok) break;
         if (lane == 0) {
-          const uint32_t st = stage_addr(k);
-          ptx::mbar_arrive_expect_tx(full_bar(k % STG), 2 * kRHalfBytes);
-          ptx::tma_load_3d(st, &p.tmap_r, full_bar(k % STG), 0, ps.c0, h);
-          ptx::tma_load_3d(st + kRHalfBytes, &p.tmap_r, full_bar(k % STG), 64, ps.c0, h);
+          const uint32_t st = kslot(k);
+          ptx::mbar_arrive_expect_tx(kfull(k % KS), 2 * KC::kRHalfBytes);
+          ptx::tma_load_3d(st, &p.tmap_r, kfull(k % KS), 0, c0, h);
+          ptx::tma_load_3d(st + KC::kRHalfBytes, &p.tmap_r, kfull(k % KS), 64, c0, h);
         }
         ++k;
       }
+      int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
+      int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
+      if (e0 < 0 || e0 >= p.num_pages) { bad_page = true; e0 = 0; }
+      if (tp.npg > 1 && (e1 < 0 || e1 >= p.num_pages)) { bad_page = true; e1 = 0; }
+      const int row0 = (e0 * p.Hkv + h) * kPage, row1 = (e1 * p.Hkv + h) * kPage;
+      // K tile into the K ring
       ok = __all_sync(0xffffffffu,
-                      ptx::mbar_wait(empty_bar(k % STG), ((k / STG) & 1) ^ 1, abort_flag, tlim));
+                      ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
       if (!ok) break;
-      const int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
-      const int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
       if (lane == 0) {
-        const uint32_t st = stage_addr(k);
-        const uint32_t fb = full_bar(k % STG);
-        ptx::mbar_arrive_expect_tx(fb, tp.npg * 4 * kPageHalfBytes);
+        const uint32_t st = kslot(k);
+        const uint32_t fb = kfull(k % KS);
+        ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
         for (int pi = 0; pi < tp.npg; ++pi) {
-          int phys = pi ? e1 : e0;
-          if (phys < 0 || phys >= p.num_pages) { bad_page = true; phys = 0; }
-          const int row = (phys * p.Hkv + h) * kPage;
+          const int row = pi ? row1 : row0;
           ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
           ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
-          ptx::tma_load_2d(st + 2 * kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
-          ptx::tma_load_2d(st + 3 * kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
+        }
+      }
+      ++k;
+      // V tile into the V ring
+      ok = __all_sync(0xffffffffu,
+                      ptx::mbar_wait(vempty(ti % VS), ((ti / VS) & 1) ^ 1, abort_flag, tlim));
+      if (!ok) break;
+      if (lane == 0) {
+        const uint32_t st = vslot(ti);
+        const uint32_t fb = vfull(ti % VS);
+        ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
+        for (int pi = 0; pi < tp.npg; ++pi) {
+          const int row = pi ? row1 : row0;
+          ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
+          ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
         }
         RELATTN_TRACE(0, ti);
       }
-      ++k;
+      i_v = ti + 1;
     }
     if (lane == 0) {
       if (bad_page) atomicOr(p.status, kStatusBadSeq);
       if (!ok) {
         // Let the copies already issued land before the CTA's memory is released.
         volatile int never = 0;
-        for (int kk = max(0, k - STG); kk < k; ++kk)
-          ptx::mbar_wait(full_bar(kk % STG), (kk / STG) & 1, &never, tlim);
+        for (int kk = max(0, k - KS); kk < k; ++kk)
+          ptx::mbar_wait(kfull(kk % KS), (kk / KS) & 1, &never, tlim);
+        for (int iv = max(0, i_v - VS); iv < i_v; ++iv)
+          ptx::mbar_wait(vfull(iv % VS), (iv / VS) & 1, &never, tlim);
       }
     }
   }
@@ -382,71 +454,70 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
-      constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, N, true, false);
-      const uint32_t tS = tmem, tX0 = tmem + 2 * N, tX1 = tmem + 3 * N, tO = tmem + 4 * N;
-      int k = 0, c = 0, i = 0, stage_prev = 0;
-      PlanState ps(p.nl);
+      constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
+      int k = 0, i = 0;                        // K-ring items, tiles issued
+      int cg[2] = {0, 0};                      // chunks issued per group
+      PlanState ps0(p.nl), ps1(p.nl);
       bool ok = true;
-      auto issue_pv = [&](int j, int stg) -> bool {
+      auto issue_pv = [&](int j) -> bool {
         if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
         if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
+        if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
         RELATTN_TRACE(3, j);
-        const uint32_t v = sbase + (uint32_t)(stg * kStageBytes) + 2 * kHalfTileBytes;
-        const uint32_t pb = sP0 + (uint32_t)((j & 1) * SL::kPBufBytes);
-        // P = P_hi + P_lo (two bf16 parts): O^T += V^T P_hi^T + V^T P_lo^T
+        const uint32_t v = vslot(j);
+        const uint32_t pb = sP0 + (uint32_t)((j & 1) * KC::kPBufBytes);
+        // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = ptx::sdesc_sw128(v + kk * 2048, kHalfTileBytes, 1024);
-            const uint64_t bd = ptx::sdesc_sw128(pb + part * SL::kOperandBytes + (kk >> 2) * (N * 128) +
-                                                 (kk & 3) * 32, 16, 1024);
-            ptx::umma_bf16(tO + (j & 1) * N, a, bd, kIdescPV, (part | kk) > 0);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = ptx::sdesc_sw128(v + kk * 2048, kHalfTileBytes, 1024);
+          const uint64_t bd = ptx::sdesc_noswz(pb + kk * (2 * 16 * 2 * N), 16 * 2 * N, 128);
+          ptx::umma_bf16(tO + (j & 1) * 2 * N, a, bd, kIdescPV, kk > 0);
         }
         ptx::umma_commit(o_full + 8u * (j & 1));
-        ptx::umma_commit(empty_bar(stg));
+        ptx::umma_commit(vempty(j % VS));
         return true;
       };
       for (int ti = 0; ti < g.ntiles; ++ti) {
-        const TilePlan tp = plan_tile(g, ti, p.ex, s_edges, ps);
-        // P.V of the previous tile releases its stage.  Issue it first unless
-        // this tile's data has already landed: a stage must never wait on a
-        // load that itself waits for that stage.
+        const int gq = (NG == 2) ? (ti & 1) : 0;
+        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, gq ? ps1 : ps0);
+        // P.V of the previous tile frees a V slot: issue it first unless this
+        // tile's K data has already landed (then S first, so softmax starts).
         bool pv_pending = i > 0;
         if (pv_pending) {
           const int kt = k + (tp.chunk ? 1 : 0);
-          if (!ptx::mbar_try_wait(full_bar(kt % STG), (kt / STG) & 1)) {
-            if (!(ok = issue_pv(i - 1, stage_prev))) break;
+          if (!ptx::mbar_try_wait(kfull(kt % KS), (kt / KS) & 1)) {
+            if (!(ok = issue_pv(i - 1))) break;
             pv_pending = false;
           }
         }
         if (tp.chunk) {
-          ok = ptx::mbar_wait(full_bar(k % STG), (k / STG) & 1, abort_flag, tlim) &&
-               ptx::mbar_wait(x_empty, (c & 1) ^ 1, abort_flag, tlim);
+          const int c = cg[gq];
+          ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
+               ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t st = stage_addr(k);
+          const uint32_t st = kslot(k);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * kRHalfBytes + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32;
             const uint64_t bq = ptx::sdesc_sw128(sQ + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            ptx::umma_bf16(tX0, ptx::sdesc_sw128(st + koff, 16, 1024), bq, kIdescQK, kk > 0);
-            ptx::umma_bf16(tX1, ptx::sdesc_sw128(st + 1024 + koff, 16, 1024), bq, kIdescQK, kk > 0);
+            ptx::umma_bf16(tX(gq), ptx::sdesc_sw128(st + koff, 16, 1024), bq, kIdescQK, kk > 0);
+            if constexpr (ROWS > 128)
+              ptx::umma_bf16(tX(gq) + N, ptx::sdesc_sw128(st + 1024 + koff, 16, 1024), bq, kIdescQK, kk > 0);
           }
-          ptx::umma_commit(x_full);
-          ptx::umma_commit(empty_bar(k % STG));
+          ptx::umma_commit(x_full + 8u * gq);
+          ptx::umma_commit(kempty(k % KS));
           ++k;
-          ++c;
+          cg[gq] = c + 1;
         }
-        ok = ptx::mbar_wait(full_bar(k % STG), (k / STG) & 1, abort_flag, tlim) &&
+        ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
              ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
         if (!ok) break;
         ptx::tc_fence_after();
         RELATTN_TRACE(1, i);
         {
-          const uint32_t st = stage_addr(k);
+          const uint32_t st = kslot(k);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t a = ptx::sdesc_sw128(st + (kk >> 2) * kHalfTileBytes + (kk & 3) * 32, 16, 1024);
@@ -454,13 +525,13 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::umma_bf16(tS + (i & 1) * N, a, bq, kIdescQK, kk > 0);
           }
           ptx::umma_commit(s_full + 8u * (i & 1));
+          ptx::umma_commit(kempty(k % KS));      // the K slot is free once S is done
         }
-        if (pv_pending && !(ok = issue_pv(i - 1, stage_prev))) break;
-        stage_prev = k % STG;
+        if (pv_pending && !(ok = issue_pv(i - 1))) break;
         ++k;
         ++i;
       }
-      if (ok && i > 0) ok = issue_pv(i - 1, stage_prev);
+      if (ok && i > 0) ok = issue_pv(i - 1);
       // every MMA issued so far must finish before tensor memory is released
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
@@ -470,67 +541,90 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   }
   // --------------------------------------------------------------- softmax
   else {
+    const int grp = (NG == 2) ? (warp - 2) >> 2 : 0;   // softmax group of this warp
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
     const int kl = sp * 32 + lane;            // key lane (S^T) / head-dim lane (O^T)
-    const int wsm = warp - 2;
+    const int wsm = (warp - 2) & 3;           // warp index inside the group
+    const int bar_id = 1 + grp;
     const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-    const uint32_t tS = tmem + lane_off, tX0 = tmem + 2 * N + lane_off,
-                   tX1 = tmem + 3 * N + lane_off, tO = tmem + 4 * N + lane_off;
-    float l_part[N], o_acc[N];
+    float* Y = reinterpret_cast<float*>(smem + KC::oY + grp * KC::kYBytes);
+    float* red = reinterpret_cast<float*>(smem + KC::oRed) + grp * 2 * 4 * N;
+    float* lred = reinterpret_cast<float*>(smem + KC::oLred) + grp * 4 * N;
+    float* alpha_buf = reinterpret_cast<float*>(smem + KC::oAlpha) + grp * 2 * N;
+    const uint32_t tXg = tX(grp) + lane_off;
+    // per-row running state: l (this thread's keys), O (this thread's head-dim
+    // lane), reference max; alpha_r carries this tile's rescale factors when
+    // O is taken right away (two groups)
+    float l_part[N], o_acc[N], m_ref[N];
+    float alpha_r[NG == 2 ? N : 1];
 #pragma unroll
-    for (int n = 0; n < N; ++n) { l_part[n] = 0.f; o_acc[n] = 0.f; }
-    int k = 0, c = 0, i = 0;
-    PlanState ps(p.nl);
+    for (int n = 0; n < N; ++n) { l_part[n] = 0.f; o_acc[n] = 0.f; m_ref[n] = -INFINITY; }
+#pragma unroll
+    for (int n = 0; n < (NG == 2 ? N : 1); ++n) alpha_r[n] = 1.f;
+    int c = 0, li = 0;                        // own chunks, own tiles
+    PlanState ps0(p.nl), ps1(p.nl);
     bool failed = false, aborted = false;
 
-    auto process_o = [&](int j) {
+    // Accumulate the O^T tile of tile j (this thread's head-dim lane) with
+    // the rescale factors `al` of that tile.
+    auto process_o = [&](int j, const float* al) {
       float ov[N];
       const bool okw = ptx::mbar_wait(o_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
+        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N;
 #pragma unroll
-        for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tO + (j & 1) * N + q16 * 16, ov + q16 * 16);
-        ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-      }
-      ptx::mbar_arrive(o_empty + 8u * (j & 1));
-      if (!okw) { failed = true; return; }
-      const float* al = alpha_buf + (j & 1) * N;
+        for (int part = 0; part < 2; ++part) {          // O^T from P_hi, then from P_lo
 #pragma unroll
-      for (int n = 0; n < N; ++n)
-        if (n < NQ) o_acc[n] = fmaf(o_acc[n], al[n], ov[n]);
-    };
-
-    for (int ti = 0; ti < g.ntiles; ++ti) {
-      const TilePlan tp = plan_tile(g, ti, p.ex, s_edges, ps);
-      if (tp.chunk) {
-        const bool okw = ptx::mbar_wait(x_full, c & 1, abort_flag, tlim);
-        if (okw) {
-          float xv[N];
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tX0 + q16 * 16, xv + q16 * 16);
+          for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(ob + part * N + q16 * 16, ov + q16 * 16);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int n = 0; n < N; ++n)
-            if (n < NQ) Y[kl * YS + n] = xv[n];
-          if (sp == 3) {                       // rows 128..135 come from lanes 120..127 of X1
-#pragma unroll
-            for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tX1 + q16 * 16, xv + q16 * 16);
-            ptx::tmem_wait_ld();
-            if (lane >= 24) {
-#pragma unroll
-              for (int n = 0; n < N; ++n)
-                if (n < NQ) Y[(kl + 8) * YS + n] = xv[n];
-            }
-          }
-          ptx::tc_fence_before();
+            if (n < NQ) o_acc[n] = part ? o_acc[n] + ov[n] : fmaf(o_acc[n], al[n], ov[n]);
         }
-        ptx::mbar_arrive(x_empty);
-        ++k;
-        ++c;
-        if (ptx::bar_sync_or(1, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
+        ptx::tc_fence_before();
       }
+      ptx::mbar_arrive(o_empty + 8u * (j & 1));
+      if (!okw) failed = true;
+    };
+
+    int last_tile = -1;
+    for (int ti = 0; ti < g.ntiles; ++ti) {
+      const int owner = (NG == 2) ? (ti & 1) : 0;
+      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, owner ? ps1 : ps0);
+      const int c0 = owner ? ps1.c0 : ps0.c0;
+      if (tp.chunk) {
+        if (owner == grp) {
+          // ---- new relative-row chunk: X^T (136 rows x N) -> gather table Y
+          const bool okw = ptx::mbar_wait(x_full + 8u * grp, c & 1, abort_flag, tlim);
+          if (okw) {
+            float xv[N];
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tXg + q16 * 16, xv + q16 * 16);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int n = 0; n < N; ++n)
+              if (n < NQ) Y[kl * YS + n] = xv[n];
+            if (ROWS > 128 && sp == 3) {         // rows 128..135 come from lanes 120..127 of X1
+#pragma unroll
+              for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tXg + N + q16 * 16, xv + q16 * 16);
+              ptx::tmem_wait_ld();
+              if (lane >= 24) {
+#pragma unroll
+                for (int n = 0; n < N; ++n)
+                  if (n < NQ) Y[(kl + 8) * YS + n] = xv[n];
+              }
+            }
+            ptx::tc_fence_before();
+          }
+          ptx::mbar_arrive(x_empty + 8u * grp);
+          ++c;
+          if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
+        }
+      }
+      if (owner != grp) continue;
+      const int i = ti;                       // buffers and phases follow the tile index
 
       // ---- S^T tile: this thread owns key j
       float s[N];
@@ -539,7 +633,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         ptx::tc_fence_after();
         RELATTN_TRACE(4, i);
 #pragma unroll
-        for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tS + (i & 1) * N + q16 * 16, s + q16 * 16);
+        for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tS + lane_off + (i & 1) * N + q16 * 16, s + q16 * 16);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
       }
@@ -555,7 +649,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
           // bucket: the distance itself below ex, else step down from the
           // tile's largest tail bucket (a tile spans only a few of them)
-          const int r = !v ? 0 : (d < p.ex ? d : p.ex + step_down(tp.k_hi, d, s_edges)) - ps.c0;
+          const int r = !v ? 0 : (d < p.ex ? d : p.ex + step_down(tp.k_hi, d, s_edges)) - c0;
           const float* yrow = Y + r * YS;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg) {
@@ -570,40 +664,76 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           }
         }
       }
-      // ---- tile max over the 128 keys
-      float* redb = red + (i & 1) * 4 * N;
+      // ---- lazy max: p = exp2(x - m_ref) with the row's reference max
+      //      m_ref.  Only when some logit exceeds it by more than kLazyLog2
+      //      (the first tile, or a jump) does the group take the tile max
+      //      and rescale; otherwise alpha = 1 and no reduction is needed.
+      //      Results stay exact: lse = m_ref + log2(l) for any m_ref.
+      bool over = false;
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (n < NQ) {
-          const float mx = warp_max(s[n]);
-          if (lane == 0) redb[wsm * N + n] = mx;
+      for (int n = 0; n < N; ++n)
+        if (n < NQ) over |= s[n] > m_ref[n] + kLazyLog2;
+      float* al_buf = alpha_buf + (li & 1) * N;
+      if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, over || !okw || failed)) {
+        if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
+        float* redb = red + (li & 1) * 4 * N;
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          if (n < NQ) {
+            const float mx = warp_max(s[n]);
+            if (lane == 0) redb[wsm * N + n] = mx;
+          }
+        }
+        ptx::bar_sync_or(bar_id, kSoftmaxThreads, false);
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          if (n < NQ) {
+            const float tmax = fmaxf(fmaxf(redb[n], redb[N + n]), fmaxf(redb[2 * N + n], redb[3 * N + n]));
+            const float mn = fmaxf(m_ref[n], tmax);
+            const float alpha = exp2f(m_ref[n] - ((mn == -INFINITY) ? 0.f : mn));
+            l_part[n] *= alpha;
+            if constexpr (NG == 2) alpha_r[n] = alpha;
+            else if (kl == 0) al_buf[n] = alpha;
+            m_ref[n] = mn;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          if constexpr (NG == 2) alpha_r[n] = 1.f;
+          else if (kl == 0 && n < NQ) al_buf[n] = 1.f;
         }
       }
-      if (ptx::bar_sync_or(1, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
       RELATTN_TRACE(5, i);
-      const float* m_old = m_buf + ((i & 1) ^ 1) * N;
-      float* m_new_buf = m_buf + (i & 1) * N;
-      float* al_buf = alpha_buf + (i & 1) * N;
-      const uint32_t pbuf = sP0 + (uint32_t)((i & 1) * SL::kPBufBytes);
-      const uint32_t p_row_base = pbuf + (uint32_t)((kl >> 6) * (N * 128));
-      const uint32_t u = (uint32_t)((kl & 63) >> 3), byte_in = (uint32_t)((kl & 7) * 2);
+      // ---- P = exp2(x - m_ref) as bf16 hi + lo parts (~16 significant bits in
+      //      the P.V product), stacked [P_hi; P_lo] = 2N rows, MN-major without
+      //      swizzle: 8-row x 16-byte core matrices, row blocks 128 B apart,
+      //      8-key groups 32*N B apart; each thread writes its key with 16-byte
+      //      stores.
+      {
+        const uint32_t pbuf = sP0 + (uint32_t)((i & 1) * KC::kPBufBytes);
+        const uint32_t prow = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16);
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (n < NQ) {
-          const float tmax = fmaxf(fmaxf(redb[n], redb[N + n]), fmaxf(redb[2 * N + n], redb[3 * N + n]));
-          const float mo = m_old[n];
-          const float mn = fmaxf(mo, tmax);
-          const float mu = (mn == -INFINITY) ? 0.f : mn;
-          const float alpha = exp2f(mo - mu);
-          const float pv = exp2f(s[n] - mu);
-          l_part[n] = fmaf(l_part[n], alpha, pv);
-          if (kl == 0) { m_new_buf[n] = mn; al_buf[n] = alpha; }
-          // bf16 hi/lo split keeps ~16 significant bits of p in the P.V product
-          const __nv_bfloat16 ph = __float2bfloat16_rn(pv);
-          const __nv_bfloat16 pl = __float2bfloat16_rn(pv - __bfloat162float(ph));
-          const uint32_t addr = p_row_base + n * 128 + ((u ^ (n & 7)) << 4) + byte_in;
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(ph)) : "memory");
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr + SL::kOperandBytes), "h"(__bfloat16_as_ushort(pl)) : "memory");
+        for (int cb = 0; cb < N / 8; ++cb) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const int n0 = cb * 8 + 2 * q2, n1 = n0 + 1;
+            float p0 = 0.f, p1 = 0.f;
+            if (n0 < NQ) p0 = exp2f(s[n0] - ((m_ref[n0] == -INFINITY) ? 0.f : m_ref[n0]));
+            if (n1 < NQ) p1 = exp2f(s[n1] - ((m_ref[n1] == -INFINITY) ? 0.f : m_ref[n1]));
+            if (n0 < NQ) l_part[n0] += p0;
+            if (n1 < NQ) l_part[n1] += p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - __low2float(h2), p1 - __high2float(h2));
+            hi[q2] = *reinterpret_cast<const uint32_t*>(&h2);
+            lo[q2] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+          const uint32_t addr = prow + cb * 128;                 // rows of P_hi
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(addr), "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"    // rows N.. of P_lo
+                       ::"r"(addr + N * 16), "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
         }
       }
       // ---- keys no token may see: clear their V rows (stale or poisoned data
@@ -612,8 +742,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
         if (!any_valid) {
           volatile int never = 0;
-          ptx::mbar_wait(full_bar(k % STG), (k / STG) & 1, &never, tlim);
-          uint8_t* vrow = smem + (k % STG) * kStageBytes + 2 * kHalfTileBytes + kl * 128;
+          ptx::mbar_wait(vfull(i % VS), (i / VS) & 1, &never, tlim);
+          uint8_t* vrow = smem + KC::oV + (i % VS) * kVSlotBytes + kl * 128;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             reinterpret_cast<uint4*>(vrow)[q] = make_uint4(0, 0, 0, 0);
@@ -624,20 +754,30 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
       RELATTN_TRACE(6, i);
-      if (i > 0) {
-        process_o(i - 1);
-        RELATTN_TRACE(7, i - 1);
+      if constexpr (NG == 2) {
+        // this group's next tile is i + 2: take O(i) now
+        process_o(i, alpha_r);
+        RELATTN_TRACE(7, i);
+      } else {
+        if (last_tile >= 0) {
+          process_o(last_tile, alpha_buf + ((li - 1) & 1) * N);
+          RELATTN_TRACE(7, last_tile);
+        }
       }
-      ++k;
-      ++i;
+      last_tile = i;
+      ++li;
     }
-    if (!aborted) {
-      if (ptx::bar_sync_or(1, kSoftmaxThreads, failed)) aborted = true;
-      else process_o(i - 1);
+    if constexpr (NG == 1) {
+      if (!aborted) {
+        if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, failed)) aborted = true;
+        else if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * N);
+      }
     }
     ptx::pdl_launch_dependents();
+
+    // ---- epilogue: finish l inside the group
+    bool bad = aborted || failed;
     if (!aborted) {
-      // ---- epilogue: finish l, normalise, write this split's rows
 #pragma unroll
       for (int n = 0; n < N; ++n) {
         if (n < NQ) {
@@ -645,27 +785,67 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           if (lane == 0) lred[wsm * N + n] = sum;
         }
       }
-      if (ptx::bar_sync_or(1, kSoftmaxThreads, failed)) aborted = true;
-      if (!aborted) {
-        const float* m_fin = m_buf + ((i - 1) & 1) * N;
-        const int rows = p.B * T * p.Hq;
-        const int d = kl;
+      if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, failed)) bad = true;
+    }
+    // l_part now holds the group's total l per row, o_acc its unnormalised O
+    float m_row[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+      if (n < NQ) {
+        l_part[n] = (li > 0 && !bad) ? lred[n] + lred[N + n] + lred[2 * N + n] + lred[3 * N + n] : 0.f;
+        m_row[n] = (li > 0 && !bad) ? m_ref[n] : -INFINITY;
+      }
+    }
+    if constexpr (NG == 2) {
+      // ---- merge group 1's state into group 0 (through the now idle K slots;
+      //      the first barrier guarantees every P.V has finished reading them)
+      bad = ptx::bar_sync_or(3, 2 * kSoftmaxThreads, bad);
+      float* xo = reinterpret_cast<float*>(smem);            // [N][128]
+      float* xm = xo + N * kHeadDim;                          // [N]
+      float* xl = xm + N;                                     // [N]
+      if (grp == 1 && !bad) {
 #pragma unroll
         for (int n = 0; n < N; ++n) {
           if (n < NQ) {
-            const int t = n / G, gg = n % G;
-            const int row = (b * T + t) * p.Hq + h * G + gg;
-            const float lt = lred[n] + lred[N + n] + lred[2 * N + n] + lred[3 * N + n];
-            const float o = (lt > 0.f) ? o_acc[n] / lt : 0.f;
-            const float lse_v = (lt > 0.f) ? (m_fin[n] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-            if (p.num_splits == 1) {
-              if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
-              else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
-              if (p.lse && d == 0) p.lse[row] = lse_v;
-            } else {
-              p.ws_o[((size_t)s_idx * rows + row) * kHeadDim + d] = o;
-              if (d == 0) p.ws_lse[(size_t)s_idx * rows + row] = lse_v;
-            }
+            xo[n * kHeadDim + kl] = o_acc[n];
+            if (kl == 0) { xm[n] = m_row[n]; xl[n] = l_part[n]; }
+          }
+        }
+      }
+      bad = ptx::bar_sync_or(3, 2 * kSoftmaxThreads, bad);
+      if (grp == 0 && !bad) {
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          if (n < NQ) {
+            const float m1 = xm[n];
+            const float m = fmaxf(m_row[n], m1);
+            const float mu = (m == -INFINITY) ? 0.f : m;
+            const float s0 = exp2f(m_row[n] - mu), s1 = exp2f(m1 - mu);
+            o_acc[n] = o_acc[n] * s0 + xo[n * kHeadDim + kl] * s1;
+            l_part[n] = l_part[n] * s0 + xl[n] * s1;
+            m_row[n] = m;
+          }
+        }
+      }
+    }
+    if (grp == 0 && !bad) {
+      const int rows = p.B * T * p.Hq;
+      const int d = kl;
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        if (n < NQ) {
+          const int t = n / G, gg = n % G;
+          const int row = (b * T + t) * p.Hq + h * G + gg;
+          const float lt = l_part[n];
+          const float o = (lt > 0.f) ? o_acc[n] / lt : 0.f;
+          const float lse_v = (lt > 0.f) ? (m_row[n] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+          if (p.num_splits == 1) {
+            if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
+            else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
+            if (p.lse && d == 0) p.lse[row] = lse_v;
+          } else {
+            p.ws_o[((size_t)s_idx * rows + row) * kHeadDim + d] = o;
+            if (d == 0) p.ws_lse[(size_t)s_idx * rows + row] = lse_v;
           }
         }
       }
@@ -676,9 +856,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   ptx::tc_fence_before();
   __syncthreads();
   if (tid == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);
+  RELATTN_TRACE(17, 0);
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, SL::kTmemCols);
+    ptx::tmem_dealloc(tmem, KC::kTmemCols);
   }
 }
 
