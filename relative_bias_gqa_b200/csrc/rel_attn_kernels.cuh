@@ -95,8 +95,9 @@ struct KernelConfig {
   static constexpr int kRows = (N == 16) ? 128 : 136;
   static constexpr int kRHalfBytes = kRows * 128;
   static constexpr int kKSlotBytes = 2 * kRHalfBytes;          // >= one K tile (32 KB)
-  static constexpr int kKSlots = 2;
-  static constexpr int kVSlots = (N == 16) ? 4 : (N == 32 ? 3 : 2);
+  static constexpr int kKSlots = (N == 16) ? 3 : 2;
+  static constexpr int kVSlots = (N == 16) ? 3 : (N == 32 ? 3 : 2);
+  static constexpr int kVLag = (N == 16) ? 1 : 0;               // V issued this many tiles after K
   // Relative-table gather stride: odd for conflict-free gathers.  The N = 16
   // instance serves at most 6 live rows.
   static constexpr int kYStride = (N == 16) ? 7 : N + 1;
@@ -310,60 +311,65 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
-  if (warp == 0) {
-    if (lane == 0) {
-      for (int s = 0; s < KS; ++s) {
-        ptx::mbar_init(kfull(s), 1);
-        ptx::mbar_init(kempty(s), 1);
-      }
-      for (int s = 0; s < VS; ++s) {
-        ptx::mbar_init(vfull(s), 1);
-        ptx::mbar_init(vempty(s), 1);
-      }
-      for (int i = 0; i < 2; ++i) {
-        ptx::mbar_init(s_full + 8u * i, 1);
-        ptx::mbar_init(s_empty + 8u * i, kSoftmaxThreads);
-        ptx::mbar_init(p_full + 8u * i, kSoftmaxThreads);
-        ptx::mbar_init(o_full + 8u * i, 1);
-        ptx::mbar_init(o_empty + 8u * i, kSoftmaxThreads);
-      }
-      for (int gq = 0; gq < NG; ++gq) {
-        ptx::mbar_init(x_full + 8u * gq, 1);
-        ptx::mbar_init(x_empty + 8u * gq, kSoftmaxThreads);
-      }
-      ptx::mbar_init(drain_bar, 1);
-      *abort_flag = 0;
-      ptx::fence_mbar_init();
-      ptx::prefetch_tmap(&p.tmap_k);
-      ptx::prefetch_tmap(&p.tmap_v);
-      ptx::prefetch_tmap(&p.tmap_r);
+  // Barriers first; the producer starts loading right after, while the other
+  // warps allocate tensor memory and stage Q and the bucket edges.
+  if (tid == 0) {
+    for (int s = 0; s < KS; ++s) {
+      ptx::mbar_init(kfull(s), 1);
+      ptx::mbar_init(kempty(s), 1);
     }
-  } else if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), KC::kTmemCols);
-    ptx::tmem_relinquish();
-  } else {
-    const int st = tid - 64;
-    const int nst = kSoftmaxThreads * NG;
-    // Q group tile: rows n = t*G + g (padding rows zero), 128B-swizzled K-major.
-    for (int u = st; u < N * 16; u += nst) {
-      const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n < NQ) {
-        const int t = n / G, gg = n % G;
-        const __nv_bfloat16* src = p.q + ((size_t)(b * T + t) * p.Hq + h * G + gg) * kHeadDim
-                                   + half * 64 + w16 * 8;
-        v = __ldg(reinterpret_cast<const uint4*>(src));
-      }
-      uint8_t* dst = smem + KC::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = v;
+    for (int s = 0; s < VS; ++s) {
+      ptx::mbar_init(vfull(s), 1);
+      ptx::mbar_init(vempty(s), 1);
     }
-    for (int e = st; e <= p.nl; e += nst) s_edges[e] = p.edges[e];
-    ptx::fence_proxy_async_smem();
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(s_full + 8u * i, 1);
+      ptx::mbar_init(s_empty + 8u * i, kSoftmaxThreads);
+      ptx::mbar_init(p_full + 8u * i, kSoftmaxThreads);
+      ptx::mbar_init(o_full + 8u * i, 1);
+      ptx::mbar_init(o_empty + 8u * i, kSoftmaxThreads);
+    }
+    for (int gq = 0; gq < NG; ++gq) {
+      ptx::mbar_init(x_full + 8u * gq, 1);
+      ptx::mbar_init(x_empty + 8u * gq, kSoftmaxThreads);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&p.tmap_k);
+    ptx::prefetch_tmap(&p.tmap_v);
+    ptx::prefetch_tmap(&p.tmap_r);
   }
-  ptx::tc_fence_before();
   __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  uint32_t tmem = 0;
+  if (warp != 0) {
+    if (warp == 1) {
+      ptx::tmem_alloc(ptx::smem_addr(tmem_holder), KC::kTmemCols);
+      ptx::tmem_relinquish();
+    } else {
+      const int st = tid - 64;
+      const int nst = kSoftmaxThreads * NG;
+      // Q group tile: rows n = t*G + g (padding rows zero), 128B-swizzled K-major.
+      for (int u = st; u < N * 16; u += nst) {
+        const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < NQ) {
+          const int t = n / G, gg = n % G;
+          const __nv_bfloat16* src = p.q + ((size_t)(b * T + t) * p.Hq + h * G + gg) * kHeadDim
+                                     + half * 64 + w16 * 8;
+          v = __ldg(reinterpret_cast<const uint4*>(src));
+        }
+        uint8_t* dst = smem + KC::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = v;
+      }
+      for (int e = st; e <= p.nl; e += nst) s_edges[e] = p.edges[e];
+      ptx::fence_proxy_async_smem();
+    }
+    ptx::tc_fence_before();
+    ptx::bar_sync_or(4, KC::kThreads - 32, false);   // every warp but the producer
+    ptx::tc_fence_after();
+    tmem = *tmem_holder;
+  }
   const uint32_t tS = tmem, tO = tmem + 2 * N;                         // O buffer b at +2N*b
   auto tX = [&](int gq) { return tmem + 6 * N + KC::kXCols * gq; };   // X0; X1 at +N
 
@@ -379,64 +385,74 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     int bt_next = bt_load(1);
     int k = 0;                                // K-ring items issued
     int i_v = 0;                              // V-ring items (= tiles) issued
+    int rows0[2] = {0, 0}, rows1[2] = {0, 0}, npgs[2] = {0, 0};
     PlanState ps0(p.nl), ps1(p.nl);
     bool ok = true, bad_page = false;
-    for (int ti = 0; ti < g.ntiles; ++ti) {
-      if (ti > 0 && (ti & 15) == 0) {
-        bt_cur = bt_next;
-        bt_next = bt_load((ti >> 4) + 1);
-      }
-      const bool odd = (NG == 2) && (ti & 1);
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, odd ? ps1 : ps0);
-      const int c0 = odd ? ps1.c0 : ps0.c0;
-      if (tp.chunk) {
+    // V of tile t is issued kVLag tiles after K of tile t, so a V slot is not
+    // held while the tile's S and softmax run.
+    for (int ti = 0; ti < g.ntiles + KC::kVLag; ++ti) {
+      if (ti < g.ntiles) {
+        if (ti > 0 && (ti & 15) == 0) {
+          bt_cur = bt_next;
+          bt_next = bt_load((ti >> 4) + 1);
+        }
+        const bool odd = (NG == 2) && (ti & 1);
+        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.edges, odd ? ps1 : ps0);
+        const int c0 = odd ? ps1.c0 : ps0.c0;
+        if (tp.chunk) {
+          ok = __all_sync(0xffffffffu,
+                          ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
+          if (!ok) break;
+          if (lane == 0) {
+            const uint32_t st = kslot(k);
+            ptx::mbar_arrive_expect_tx(kfull(k % KS), 2 * KC::kRHalfBytes);
+            ptx::tma_load_3d(st, &p.tmap_r, kfull(k % KS), 0, c0, h);
+            ptx::tma_load_3d(st + KC::kRHalfBytes, &p.tmap_r, kfull(k % KS), 64, c0, h);
+          }
+          ++k;
+        }
+        int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
+        int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
+        if (e0 < 0 || e0 >= p.num_pages) { bad_page = true; e0 = 0; }
+        if (tp.npg > 1 && (e1 < 0 || e1 >= p.num_pages)) { bad_page = true; e1 = 0; }
+        rows0[ti & 1] = (e0 * p.Hkv + h) * kPage;
+        rows1[ti & 1] = (e1 * p.Hkv + h) * kPage;
+        npgs[ti & 1] = tp.npg;
+        // K tile into the K ring
         ok = __all_sync(0xffffffffu,
                         ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
         if (!ok) break;
         if (lane == 0) {
           const uint32_t st = kslot(k);
-          ptx::mbar_arrive_expect_tx(kfull(k % KS), 2 * KC::kRHalfBytes);
-          ptx::tma_load_3d(st, &p.tmap_r, kfull(k % KS), 0, c0, h);
-          ptx::tma_load_3d(st + KC::kRHalfBytes, &p.tmap_r, kfull(k % KS), 64, c0, h);
+          const uint32_t fb = kfull(k % KS);
+          ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
+          for (int pi = 0; pi < tp.npg; ++pi) {
+            const int row = pi ? rows1[ti & 1] : rows0[ti & 1];
+            ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
+            ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
+          }
         }
         ++k;
       }
-      int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
-      int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
-      if (e0 < 0 || e0 >= p.num_pages) { bad_page = true; e0 = 0; }
-      if (tp.npg > 1 && (e1 < 0 || e1 >= p.num_pages)) { bad_page = true; e1 = 0; }
-      const int row0 = (e0 * p.Hkv + h) * kPage, row1 = (e1 * p.Hkv + h) * kPage;
-      // K tile into the K ring
-      ok = __all_sync(0xffffffffu,
-                      ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
-      if (!ok) break;
-      if (lane == 0) {
-        const uint32_t st = kslot(k);
-        const uint32_t fb = kfull(k % KS);
-        ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
-        for (int pi = 0; pi < tp.npg; ++pi) {
-          const int row = pi ? row1 : row0;
-          ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
-          ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
+      const int tv = ti - KC::kVLag;
+      if (tv >= 0 && tv < g.ntiles) {
+        // V tile into the V ring
+        ok = __all_sync(0xffffffffu,
+                        ptx::mbar_wait(vempty(tv % VS), ((tv / VS) & 1) ^ 1, abort_flag, tlim));
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t st = vslot(tv);
+          const uint32_t fb = vfull(tv % VS);
+          ptx::mbar_arrive_expect_tx(fb, npgs[tv & 1] * 2 * kPageHalfBytes);
+          for (int pi = 0; pi < npgs[tv & 1]; ++pi) {
+            const int row = pi ? rows1[tv & 1] : rows0[tv & 1];
+            ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
+            ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
+          }
+          RELATTN_TRACE(0, tv);
         }
+        i_v = tv + 1;
       }
-      ++k;
-      // V tile into the V ring
-      ok = __all_sync(0xffffffffu,
-                      ptx::mbar_wait(vempty(ti % VS), ((ti / VS) & 1) ^ 1, abort_flag, tlim));
-      if (!ok) break;
-      if (lane == 0) {
-        const uint32_t st = vslot(ti);
-        const uint32_t fb = vfull(ti % VS);
-        ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
-        for (int pi = 0; pi < tp.npg; ++pi) {
-          const int row = pi ? row1 : row0;
-          ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
-          ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
-        }
-        RELATTN_TRACE(0, ti);
-      }
-      i_v = ti + 1;
     }
     if (lane == 0) {
       if (bad_page) atomicOr(p.status, kStatusBadSeq);
@@ -455,6 +471,12 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     if (lane == 0) {
       constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
       constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
+      // Base descriptors; every MMA operand below is one of these plus a
+      // constant byte offset (the address field is the low 14 bits, >> 4).
+      const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
+      const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
+      const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + KC::oV, kHalfTileBytes, 1024);  // V^T, MN-major
+      const uint64_t pdesc0 = ptx::sdesc_noswz(sP0, 16 * 2 * N, 128);              // [P_hi; P_lo], MN-major
       int k = 0, i = 0;                        // K-ring items, tiles issued
       int cg[2] = {0, 0};                      // chunks issued per group
       PlanState ps0(p.nl), ps1(p.nl);
@@ -465,14 +487,13 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
         RELATTN_TRACE(3, j);
-        const uint32_t v = vslot(j);
-        const uint32_t pb = sP0 + (uint32_t)((j & 1) * KC::kPBufBytes);
+        const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
+        const uint64_t pbd = pdesc0 + (uint64_t)(((j & 1) * KC::kPBufBytes) >> 4);
         // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = ptx::sdesc_sw128(v + kk * 2048, kHalfTileBytes, 1024);
-          const uint64_t bd = ptx::sdesc_noswz(pb + kk * (2 * 16 * 2 * N), 16 * 2 * N, 128);
-          ptx::umma_bf16(tO + (j & 1) * 2 * N, a, bd, kIdescPV, kk > 0);
+          ptx::umma_bf16(tO + (j & 1) * 2 * N, va + (uint64_t)((kk * 2048) >> 4),
+                         pbd + (uint64_t)((kk * (2 * 16 * 2 * N)) >> 4), kIdescPV, kk > 0);
         }
         ptx::umma_commit(o_full + 8u * (j & 1));
         ptx::umma_commit(vempty(j % VS));
@@ -497,14 +518,14 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
                ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint32_t st = kslot(k);
+          const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32;
-            const uint64_t bq = ptx::sdesc_sw128(sQ + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            ptx::umma_bf16(tX(gq), ptx::sdesc_sw128(st + koff, 16, 1024), bq, kIdescQK, kk > 0);
+            const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
+            const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+            ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
             if constexpr (ROWS > 128)
-              ptx::umma_bf16(tX(gq) + N, ptx::sdesc_sw128(st + 1024 + koff, 16, 1024), bq, kIdescQK, kk > 0);
+              ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
           }
           ptx::umma_commit(x_full + 8u * gq);
           ptx::umma_commit(kempty(k % KS));
@@ -517,12 +538,11 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         ptx::tc_fence_after();
         RELATTN_TRACE(1, i);
         {
-          const uint32_t st = kslot(k);
+          const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = ptx::sdesc_sw128(st + (kk >> 2) * kHalfTileBytes + (kk & 3) * 32, 16, 1024);
-            const uint64_t bq = ptx::sdesc_sw128(sQ + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            ptx::umma_bf16(tS + (i & 1) * N, a, bq, kIdescQK, kk > 0);
+            ptx::umma_bf16(tS + (i & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
+                           qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
           }
           ptx::umma_commit(s_full + 8u * (i & 1));
           ptx::umma_commit(kempty(k % KS));      // the K slot is free once S is done
@@ -642,14 +662,26 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       const int j = tp.j0 + kl;
       const bool loaded = kl < tp.npg * kPage;
       const int d0 = g.p0 - j;                    // distance from token 0
+      // The tile's tail buckets lie just below k_hi (log buckets are at least
+      // 28 keys wide, so a 128-key tile spans at most a few): the four edges
+      // below it, loaded once per tile, place almost every key by compares.
+      int e_hi[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) e_hi[m] = s_edges[max(tp.k_hi - m, 0)];
 #pragma unroll
       for (int t = 0; t < TMAX; ++t) {
         if (t < T) {
           const int d = d0 + t;
           const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
-          // bucket: the distance itself below ex, else step down from the
-          // tile's largest tail bucket (a tile spans only a few of them)
-          const int r = !v ? 0 : (d < p.ex ? d : p.ex + step_down(tp.k_hi, d, s_edges)) - c0;
+          int bk = d;                               // exact region: the distance itself
+          if (v && d >= p.ex) {
+            int k = tp.k_hi - (int)(e_hi[0] > d) - (int)(e_hi[1] > d) - (int)(e_hi[2] > d) -
+                    (int)(e_hi[3] > d);
+            k = max(k, 0);
+            if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges);
+            bk = p.ex + k;
+          }
+          const int r = v ? bk - c0 : 0;
           const float* yrow = Y + r * YS;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg) {
@@ -902,21 +934,29 @@ rel_attn_combine_kernel(const float* __restrict__ ws_lse, const float* __restric
     sum += w[q];
   }
   sum = warp_sum(sum);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // weights to shared memory, then the split outputs 8 at a time so the
+  // loads overlap instead of waiting one L2 round trip per split
+  __shared__ float wsh[4][256];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    if (q * 32 >= num_splits) break;
-    const int cnt = min(32, num_splits - q * 32);
-    for (int sl = 0; sl < cnt; ++sl) {
-      const float ws = __shfl_sync(0xffffffffu, w[q], sl);
-      if (ws != 0.f) {
-        const float4 o = __ldg(reinterpret_cast<const float4*>(
-            ws_o + ((size_t)(q * 32 + sl) * rows + row) * kHeadDim) + lane);
-        acc.x = fmaf(ws, o.x, acc.x);
-        acc.y = fmaf(ws, o.y, acc.y);
-        acc.z = fmaf(ws, o.z, acc.z);
-        acc.w = fmaf(ws, o.w, acc.w);
-      }
+  for (int q = 0; q < 8; ++q) wsh[warp][q * 32 + lane] = w[q];
+  __syncwarp();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int base = 0; base < num_splits; base += 8) {
+    float4 o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = base + u;
+      o[u] = (s < num_splits && wsh[warp][s] != 0.f)
+                 ? __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)s * rows + row) * kHeadDim) + lane)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float ws = (base + u < num_splits) ? wsh[warp][base + u] : 0.f;
+      acc.x = fmaf(ws, o[u].x, acc.x);
+      acc.y = fmaf(ws, o[u].y, acc.y);
+      acc.z = fmaf(ws, o[u].z, acc.z);
+      acc.w = fmaf(ws, o[u].w, acc.w);
     }
   }
   const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
