@@ -17,13 +17,14 @@ namespace relattn {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxQTokens = 8;         // query tokens per sequence (speculative verify)
 constexpr size_t kHeaderBytes = 256;   // status word lives here
 
 struct DeviceInfo {
   bool probed = false;
   bool sm100 = false;
   int sm_count = 0;
-  bool attr_set[4] = {false, false, false, false};
+  bool attr_set[kMaxQTokens] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -58,7 +59,7 @@ int group_width(int G, int T) {
 int validate_shape(const rel_attn_shape* s) {
   if (!s) return REL_ATTN_ERR_INVALID_ARG;
   if (s->batch < 1 || s->batch > 65535) return REL_ATTN_ERR_INVALID_ARG;
-  if (s->q_tokens < 1 || s->q_tokens > 8) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->q_tokens < 1 || s->q_tokens > kMaxQTokens) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_kv_heads < 1 || s->num_kv_heads > 65535) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_q_heads < 1 || s->num_q_heads % s->num_kv_heads) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_q_heads / s->num_kv_heads != 6) return REL_ATTN_ERR_INVALID_ARG;
@@ -223,11 +224,13 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
   return true;
 }
 
-template <int N, int NG>
-int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di,
-                   int slot) {
+template <int T>
+int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
+  constexpr int N = (6 * T <= 6) ? 16 : (6 * T <= 32 ? 32 : 48);    // group width, as group_width()
+  constexpr int NG = (N == 16) ? 2 : 1;
+  constexpr int slot = T - 1;
   using KC = KernelConfig<N, NG>;
-  auto kern = rel_attn_partial_kernel<N, 6, NG>;
+  auto kern = rel_attn_partial_kernel<N, 6, NG, T>;
   constexpr int smem = KC::kAllocBytes;
   if (!di.attr_set[slot]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -374,10 +377,16 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
 
 int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
                        DeviceInfo& di) {
-  switch (group_width(6, shape->q_tokens)) {
-    case 16: return launch_partial<16, 2>(prm, S, shape->batch, shape->num_kv_heads, st, di, 0);
-    case 32: return launch_partial<32, 1>(prm, S, shape->batch, shape->num_kv_heads, st, di, 1);
-    case 48: return launch_partial<48, 1>(prm, S, shape->batch, shape->num_kv_heads, st, di, 2);
+  const int B = shape->batch, Hkv = shape->num_kv_heads;
+  switch (shape->q_tokens) {
+    case 1: return launch_partial<1>(prm, S, B, Hkv, st, di);
+    case 2: return launch_partial<2>(prm, S, B, Hkv, st, di);
+    case 3: return launch_partial<3>(prm, S, B, Hkv, st, di);
+    case 4: return launch_partial<4>(prm, S, B, Hkv, st, di);
+    case 5: return launch_partial<5>(prm, S, B, Hkv, st, di);
+    case 6: return launch_partial<6>(prm, S, B, Hkv, st, di);
+    case 7: return launch_partial<7>(prm, S, B, Hkv, st, di);
+    case 8: return launch_partial<8>(prm, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }
@@ -392,8 +401,8 @@ int launch_combine(const rel_attn_shape* shape, int S, void* out, float* lse, vo
   const float* ws_o = reinterpret_cast<const float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)((rows + 3) / 4));
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

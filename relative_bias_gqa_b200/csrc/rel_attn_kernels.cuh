@@ -42,6 +42,14 @@
 #ifndef RELATTN_TRACE
 #define RELATTN_TRACE(event, tile)
 #endif
+// Which split / KV head a block works on (the identity unless a study build
+// permutes the placement).
+#ifndef RELATTN_SPLIT_OF_BLOCK
+#define RELATTN_SPLIT_OF_BLOCK(x) (x)
+#endif
+#ifndef RELATTN_HEAD_OF_BLOCK
+#define RELATTN_HEAD_OF_BLOCK(y) (y)
+#endif
 
 namespace relattn {
 
@@ -129,7 +137,7 @@ struct KernelConfig {
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
   static_assert(kKSlotBytes >= 2 * kHalfTileBytes && oV % 1024 == 0 && oQ % 1024 == 0,
                 "slot layout");
-  static_assert(oV >= N * 128 * 4 + 2 * N * 4, "exchange area");
+  static_assert(oV >= NG * N * 128 * 4 * 2 + NG * N * 4 * 2, "epilogue exchange area");
 };
 
 // Per-CTA geometry shared by the three roles.
@@ -237,7 +245,9 @@ __device__ void fill_rows(const DecodeParams& p, int b, int h, int s, float o_va
   }
 }
 
-template <int N, int G, int NG>
+// T (query tokens) is a template parameter: every per-row loop below runs
+// over the NQ = T*G live rows only, fully unrolled.
+template <int N, int G, int NG, int T>
 __global__ void __launch_bounds__(KernelConfig<N, NG>::kThreads, 1)
 rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   using KC = KernelConfig<N, NG>;
@@ -245,7 +255,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int VS = KC::kVSlots;
   constexpr int ROWS = KC::kRows;
   constexpr int YS = KC::kYStride;
-  constexpr int TMAX = (N + G - 1) / G;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -254,9 +263,9 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int T = p.T;
-  const int NQ = T * G;
+  const int s_idx = RELATTN_SPLIT_OF_BLOCK(blockIdx.x), h = RELATTN_HEAD_OF_BLOCK(blockIdx.y), b = blockIdx.z;
+  constexpr int NQ = T * G;
+  static_assert(NQ <= N, "group width");
   RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
@@ -569,7 +578,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
     float* Y = reinterpret_cast<float*>(smem + KC::oY + grp * KC::kYBytes);
     float* red = reinterpret_cast<float*>(smem + KC::oRed) + grp * 2 * 4 * N;
-    float* lred = reinterpret_cast<float*>(smem + KC::oLred) + grp * 4 * N;
     float* alpha_buf = reinterpret_cast<float*>(smem + KC::oAlpha) + grp * 2 * N;
     const uint32_t tXg = tX(grp) + lane_off;
     // per-row running state: l (this thread's keys), O (this thread's head-dim
@@ -609,6 +617,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     };
 
     int last_tile = -1;
+    RELATTN_TRACE(5, 63);
     for (int ti = 0; ti < g.ntiles; ++ti) {
       const int owner = (NG == 2) ? (ti & 1) : 0;
       const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, owner ? ps1 : ps0);
@@ -639,6 +648,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::tc_fence_before();
           }
           ptx::mbar_arrive(x_empty + 8u * grp);
+          if (c == 0) RELATTN_TRACE(6, 63);
           ++c;
           if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
         }
@@ -669,8 +679,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) e_hi[m] = s_edges[max(tp.k_hi - m, 0)];
 #pragma unroll
-      for (int t = 0; t < TMAX; ++t) {
-        if (t < T) {
+      for (int t = 0; t < T; ++t) {
+        {
           const int d = d0 + t;
           const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
           int bk = d;                               // exact region: the distance itself
@@ -687,12 +697,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           for (int gg = 0; gg < G; ++gg) {
             const int n = t * G + gg;
             if (n < N) s[n] = v ? (s[n] + yrow[n]) * p.scale_log2 : -INFINITY;
-          }
-        } else {
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            const int n = t * G + gg;
-            if (n < N) s[n] = -INFINITY;
           }
         }
       }
@@ -807,78 +811,61 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     }
     ptx::pdl_launch_dependents();
 
-    // ---- epilogue: finish l inside the group
-    bool bad = aborted || failed;
-    if (!aborted) {
+    // ---- epilogue: each group's unnormalised O, per-lane l and reference
+    //      max go to shared memory (the K ring, idle once every S has been
+    //      read); then all softmax threads merge the groups and write this
+    //      CTA's rows in short loops.
+    bool bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, aborted || failed);
+    float* eo = reinterpret_cast<float*>(smem);             // [NG][NQ][128]
+    float* el = eo + NG * NQ * kHeadDim;                    // [NG][NQ][128]
+    float* em = el + NG * NQ * kHeadDim;                    // [NG][NQ]
+    float* es = em + NG * NQ;                               // [NG][NQ]
+    if (!bad) {
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (n < NQ) {
-          const float sum = warp_sum(l_part[n]);
-          if (lane == 0) lred[wsm * N + n] = sum;
-        }
+      for (int n = 0; n < NQ; ++n) {
+        eo[(grp * NQ + n) * kHeadDim + kl] = o_acc[n];
+        el[(grp * NQ + n) * kHeadDim + kl] = l_part[n];
       }
-      if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, failed)) bad = true;
-    }
-    // l_part now holds the group's total l per row, o_acc its unnormalised O
-    float m_row[N];
+      if (kl == 0) {
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-      if (n < NQ) {
-        l_part[n] = (li > 0 && !bad) ? lred[n] + lred[N + n] + lred[2 * N + n] + lred[3 * N + n] : 0.f;
-        m_row[n] = (li > 0 && !bad) ? m_ref[n] : -INFINITY;
-      }
-    }
-    if constexpr (NG == 2) {
-      // ---- merge group 1's state into group 0 (through the now idle K slots;
-      //      the first barrier guarantees every P.V has finished reading them)
-      bad = ptx::bar_sync_or(3, 2 * kSoftmaxThreads, bad);
-      float* xo = reinterpret_cast<float*>(smem);            // [N][128]
-      float* xm = xo + N * kHeadDim;                          // [N]
-      float* xl = xm + N;                                     // [N]
-      if (grp == 1 && !bad) {
-#pragma unroll
-        for (int n = 0; n < N; ++n) {
-          if (n < NQ) {
-            xo[n * kHeadDim + kl] = o_acc[n];
-            if (kl == 0) { xm[n] = m_row[n]; xl[n] = l_part[n]; }
-          }
-        }
-      }
-      bad = ptx::bar_sync_or(3, 2 * kSoftmaxThreads, bad);
-      if (grp == 0 && !bad) {
-#pragma unroll
-        for (int n = 0; n < N; ++n) {
-          if (n < NQ) {
-            const float m1 = xm[n];
-            const float m = fmaxf(m_row[n], m1);
-            const float mu = (m == -INFINITY) ? 0.f : m;
-            const float s0 = exp2f(m_row[n] - mu), s1 = exp2f(m1 - mu);
-            o_acc[n] = o_acc[n] * s0 + xo[n * kHeadDim + kl] * s1;
-            l_part[n] = l_part[n] * s0 + xl[n] * s1;
-            m_row[n] = m;
-          }
-        }
+        for (int n = 0; n < NQ; ++n) em[grp * NQ + n] = m_ref[n];
       }
     }
-    if (grp == 0 && !bad) {
+    bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, bad);
+    if (!bad) {
+      const int et = tid - 64, ew = et >> 5;               // softmax thread / warp index
+      // row sums of l: one warp per (group, row)
+      for (int r = ew; r < NG * NQ; r += 4 * NG) {
+        const float* src = el + r * kHeadDim;
+        const float v = warp_sum(src[lane] + src[lane + 32] + src[lane + 64] + src[lane + 96]);
+        if (lane == 0) es[r] = v;
+      }
+      ptx::bar_sync_or(3, kSoftmaxThreads * NG, false);
       const int rows = p.B * T * p.Hq;
-      const int d = kl;
+      for (int e = et; e < NQ * kHeadDim; e += kSoftmaxThreads * NG) {
+        const int n = e / kHeadDim, d = e % kHeadDim;
+        float m = -INFINITY;
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (n < NQ) {
-          const int t = n / G, gg = n % G;
-          const int row = (b * T + t) * p.Hq + h * G + gg;
-          const float lt = l_part[n];
-          const float o = (lt > 0.f) ? o_acc[n] / lt : 0.f;
-          const float lse_v = (lt > 0.f) ? (m_row[n] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-          if (p.num_splits == 1) {
-            if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
-            else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
-            if (p.lse && d == 0) p.lse[row] = lse_v;
-          } else {
-            p.ws_o[((size_t)s_idx * rows + row) * kHeadDim + d] = o;
-            if (d == 0) p.ws_lse[(size_t)s_idx * rows + row] = lse_v;
-          }
+        for (int q = 0; q < NG; ++q) m = fmaxf(m, em[q * NQ + n]);
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int q = 0; q < NG; ++q) {
+          const float sc = exp2f(em[q * NQ + n] - mu);
+          o = fmaf(eo[(q * NQ + n) * kHeadDim + d], sc, o);
+          l = fmaf(es[q * NQ + n], sc, l);
+        }
+        o = (l > 0.f) ? o / l : 0.f;
+        const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const int t = n / G, gg = n - t * G;
+        const int row = (b * T + t) * p.Hq + h * G + gg;
+        if (p.num_splits == 1) {
+          if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
+          else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
+          if (p.lse && d == 0) p.lse[row] = lse_v;
+        } else {
+          p.ws_o[((size_t)s_idx * rows + row) * kHeadDim + d] = o;
+          if (d == 0) p.ws_lse[(size_t)s_idx * rows + row] = lse_v;
         }
       }
     }
@@ -895,83 +882,82 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   }
 }
 
-// LSE merge of per-split partial results: one warp per (b, t, hq) row.
-__global__ void __launch_bounds__(128)
+// LSE merge of per-split partial results: one CTA per (b, t, hq) row; its
+// 8 warps take every 8th split, so the merge costs about two dependent memory
+// round trips (the lse values, then the outputs) whatever the split count.
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads)
 rel_attn_combine_kernel(const float* __restrict__ ws_lse, const float* __restrict__ ws_o,
                         int num_splits, int rows, void* out, float* lse, int out_fp32) {
   ptx::pdl_wait_primary();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;
-  if (row >= rows) return;
-  float w[8];
-  float mx = -INFINITY;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int s = q * 32 + lane;
-    w[q] = (s < num_splits) ? __ldg(ws_lse + (size_t)s * rows + row) : -INFINITY;
-    mx = fmaxf(mx, w[q]);
-  }
-  bool nan_seen = false;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) nan_seen |= (w[q] != w[q]);
-  if (__any_sync(0xffffffffu, nan_seen)) {       // a rejected sequence: propagate NaN
-    const float qnan = __int_as_float(0x7fc00000);
-    if (out_fp32) {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * kHeadDim)[lane] =
-          make_float4(qnan, qnan, qnan, qnan);
-    } else {
-      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * kHeadDim)[lane] =
-          make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+  __shared__ float w_s[256];
+  __shared__ float red[8];
+  __shared__ float4 part[8][32];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int row = blockIdx.x;
+  const float l = (t < num_splits) ? __ldg(ws_lse + (size_t)t * rows + row) : -INFINITY;
+  if (__syncthreads_or(l != l)) {                  // a rejected sequence: propagate NaN
+    if (t < 32) {
+      const float qnan = __int_as_float(0x7fc00000);
+      if (out_fp32) {
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * kHeadDim)[lane] =
+            make_float4(qnan, qnan, qnan, qnan);
+      } else {
+        reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * kHeadDim)[lane] =
+            make_uint2(0x7fc07fc0u, 0x7fc07fc0u);
+      }
+      if (lse && lane == 0) lse[row] = qnan;
     }
-    if (lse && lane == 0) lse[row] = qnan;
     return;
   }
-  mx = warp_max(mx);
-  float sum = 0.f;
+  float mx = warp_max(l);
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    w[q] = (mx == -INFINITY || w[q] == -INFINITY) ? 0.f : expf(w[q] - mx);
-    sum += w[q];
-  }
-  sum = warp_sum(sum);
-  // weights to shared memory, then the split outputs 8 at a time so the
-  // loads overlap instead of waiting one L2 round trip per split
-  __shared__ float wsh[4][256];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) wsh[warp][q * 32 + lane] = w[q];
-  __syncwarp();
+  for (int q = 1; q < 8; ++q) mx = fmaxf(mx, red[q]);
+  const float w = (mx == -INFINITY || l == -INFINITY) ? 0.f : expf(l - mx);
+  w_s[t] = w;
+  float sum = warp_sum(w);
+  __syncthreads();                                   // w_s complete, red[] reads done
+  if (lane == 0) red[warp] = sum;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int base = 0; base < num_splits; base += 8) {
-    float4 o[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = base + u;
-      o[u] = (s < num_splits && wsh[warp][s] != 0.f)
-                 ? __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)s * rows + row) * kHeadDim) + lane)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float ws = (base + u < num_splits) ? wsh[warp][base + u] : 0.f;
-      acc.x = fmaf(ws, o[u].x, acc.x);
-      acc.y = fmaf(ws, o[u].y, acc.y);
-      acc.z = fmaf(ws, o[u].z, acc.z);
-      acc.w = fmaf(ws, o[u].w, acc.w);
+  for (int s = warp; s < num_splits; s += 8) {
+    const float ws = w_s[s];
+    if (ws != 0.f) {
+      const float4 o = __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)s * rows + row) * kHeadDim) + lane);
+      acc.x = fmaf(ws, o.x, acc.x);
+      acc.y = fmaf(ws, o.y, acc.y);
+      acc.z = fmaf(ws, o.z, acc.z);
+      acc.w = fmaf(ws, o.w, acc.w);
     }
   }
-  const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
-  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-  if (out_fp32) {
-    reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * kHeadDim)[lane] = acc;
-  } else {
-    __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * kHeadDim)[lane] = pk;
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    sum = red[0];
+#pragma unroll
+    for (int q = 1; q < 8; ++q) sum += red[q];
+#pragma unroll
+    for (int q = 1; q < 8; ++q) {
+      const float4 o = part[q][lane];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    if (out_fp32) {
+      reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + (size_t)row * kHeadDim)[lane] = acc;
+    } else {
+      __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * kHeadDim)[lane] = pk;
+    }
+    if (lse && lane == 0) lse[row] = (sum > 0.f) ? mx + logf(sum) : -INFINITY;
   }
-  if (lse && lane == 0) lse[row] = (sum > 0.f) ? mx + logf(sum) : -INFINITY;
 }
 
 }  // namespace relattn

@@ -73,6 +73,11 @@ SMALL = [
     dict(L=1500, window=1), dict(L=1500, window=64), dict(L=2500, window=1024),
     dict(L=2500, T=8, window=1024, NB=1024), dict(L=3000, T=4, window=100),
     dict(L=900, NB=8), dict(L=2000, NB=1030), dict(L=200, window=1024, NB=1024),
+    # other bucket geometries: a short exact range with dense (repeated) tail
+    # edges, and distances past max_distance clamped into the last bucket
+    dict(L=6000, NB=364, exact_buckets=64, max_distance=5000),
+    dict(L=3000, T=8, NB=200, exact_buckets=16, max_distance=100000),
+    dict(L=2200, T=2, NB=600, exact_buckets=100, max_distance=1500),
 ]
 
 
