@@ -81,18 +81,26 @@ int validate_shape(const rel_attn_shape* s) {
 // Lower edges of the tail buckets.  e_k = ceil(E * (Dmax/E)^(k/NL)) in long
 // double; a value within 1e-9 (relative) of an integer is taken as that
 // integer so that exact powers (e.g. 1024 * 2^5) do not round up.
-void bucket_table(const rel_attn_shape* s, int* ex, int* nl, int* edges) {
+// `log_scale` = NL / log2(Dmax/E): (log2(d) - log2(E)) * log_scale is the
+// tail bucket of d up to rounding, a starting guess the kernels correct
+// against the table (0 when there is a single tail bucket).
+void bucket_table(const rel_attn_shape* s, int* ex, int* nl, int* edges, float* log2_ex,
+                  float* log_scale) {
   const int NB = s->num_buckets, E = s->exact_buckets;
   if (NB <= E) {
     *ex = NB - 1;
     *nl = 1;
     edges[0] = NB - 1;
+    *log2_ex = 0.f;
+    *log_scale = 0.f;
     return;
   }
   const int n = NB - E;
   *ex = E;
   *nl = n;
   const long double lr = log2l((long double)s->max_distance / (long double)E);
+  *log2_ex = (float)log2l((long double)E);
+  *log_scale = (float)((long double)n / lr);
   for (int k = 0; k <= n; ++k) {
     const long double x = (long double)E * exp2l(lr * (long double)k / (long double)n);
     const long double r = nearbyintl(x);
@@ -103,7 +111,11 @@ void bucket_table(const rel_attn_shape* s, int* ex, int* nl, int* edges) {
 
 // Small caches: the edge table depends only on (NB, E, Dmax) and a tensor
 // map only on (base pointer, extents); both are rebuilt otherwise per call.
-struct EdgeEntry { int nb = -1, e = -1, dmax = -1, ex = 0, nl = 0; int edges[kMaxTailBuckets + 1]; };
+struct EdgeEntry {
+  int nb = -1, e = -1, dmax = -1, ex = 0, nl = 0;
+  float log2_ex = 0.f, log_scale = 0.f;
+  int edges[kMaxTailBuckets + 1];
+};
 struct MapEntry { const void* base = nullptr; uint64_t a = 0, b = 0; int kind = -1; CUtensorMap map; };
 constexpr int kEdgeCache = 4, kMapCache = 16;
 EdgeEntry g_edge_cache[kEdgeCache];
@@ -111,22 +123,27 @@ MapEntry g_map_cache[kMapCache];
 int g_edge_next = 0, g_map_next = 0;
 std::mutex g_cache_mu;
 
-void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges) {
+void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges,
+                         float* log2_ex = nullptr, float* log_scale = nullptr) {
   std::lock_guard<std::mutex> lk(g_cache_mu);
+  const EdgeEntry* hit = nullptr;
   for (auto& e : g_edge_cache) {
     if (e.nb == s->num_buckets && e.e == s->exact_buckets && e.dmax == s->max_distance) {
-      *ex = e.ex;
-      *nl = e.nl;
-      memcpy(edges, e.edges, sizeof(int) * (e.nl + 1));
-      return;
+      hit = &e;
+      break;
     }
   }
-  EdgeEntry& e = g_edge_cache[g_edge_next++ % kEdgeCache];
-  bucket_table(s, &e.ex, &e.nl, e.edges);
-  e.nb = s->num_buckets; e.e = s->exact_buckets; e.dmax = s->max_distance;
-  *ex = e.ex;
-  *nl = e.nl;
-  memcpy(edges, e.edges, sizeof(int) * (e.nl + 1));
+  if (!hit) {
+    EdgeEntry& e = g_edge_cache[g_edge_next++ % kEdgeCache];
+    bucket_table(s, &e.ex, &e.nl, e.edges, &e.log2_ex, &e.log_scale);
+    e.nb = s->num_buckets; e.e = s->exact_buckets; e.dmax = s->max_distance;
+    hit = &e;
+  }
+  *ex = hit->ex;
+  *nl = hit->nl;
+  if (log2_ex) *log2_ex = hit->log2_ex;
+  if (log_scale) *log_scale = hit->log_scale;
+  memcpy(edges, hit->edges, sizeof(int) * (hit->nl + 1));
 }
 
 int bucket_host(int d, int ex, int nl, const int* edges) {
@@ -368,7 +385,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->num_splits = S;
   prm->window = window;
   prm->out_fp32 = shape->out_fp32;
-  bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges);
+  bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges, &prm->log2_ex, &prm->log_scale);
   prm->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
   *S_out = S;
   *di_out = &di;

@@ -85,6 +85,7 @@ struct alignas(64) DecodeParams {
   int ex;               // distances d < ex are their own bucket
   int nl;               // tail buckets: bucket = ex + max{k < nl : edges[k] <= d}
   float scale_log2;     // log2(e) / sqrt(D)
+  float log2_ex, log_scale;  // tail-bucket guess: (log2(d) - log2_ex) * log_scale
   int edges[kMaxTailBuckets + 1];
 };
 
@@ -163,15 +164,25 @@ struct PlanState {
   __device__ explicit PlanState(int nl) : k_hi(nl - 1), k_lo(nl - 1) {}
 };
 
-// Largest k' <= k with edges[k'] <= d (edges[0] <= d is guaranteed): a few
-// linear steps, then a binary search for long moves.
-__device__ __forceinline__ int step_down(int k, int d, const int* edges) {
-#pragma unroll 1
-  for (int s = 0; s < 4; ++s) {
-    if (k == 0 || edges[k] <= d) return k;
-    --k;
+// Largest k' <= k with edges[k'] <= d (edges[0] <= d is guaranteed).  The
+// edges grow geometrically, so (log2(d) - log2_ex) * log_scale names the
+// bucket up to rounding: the guess is checked against the table (one round of
+// independent loads) and a binary search settles anything it does not pin.
+__device__ __forceinline__ int seek_bucket(int k, int d, const int* edges, float log2_ex,
+                                           float log_scale) {
+  const float t = (__log2f((float)d) - log2_ex) * log_scale;
+  int g = (t > 0.f) ? (int)fminf(t, 65536.f) : 0;         // NaN and negatives give 0
+  g = min(g, k);
+  const int em = edges[max(g - 1, 0)], e0 = edges[g];
+  const int e1 = edges[min(g + 1, k)], e2 = edges[min(g + 2, k)];
+  if (e0 <= d) {
+    if (g == k || e1 > d) return g;
+    if (g + 1 == k || e2 > d) return g + 1;
+  } else if (g > 0 && em <= d) {
+    return g - 1;
   }
   int lo = 0, hi = k;
+#pragma unroll 1
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (edges[mid] <= d) lo = mid; else hi = mid - 1;
@@ -179,12 +190,21 @@ __device__ __forceinline__ int step_down(int k, int d, const int* edges) {
   return lo;
 }
 
+// Moves cursor k down to the tail bucket of d (d never lies above the
+// cursor's bucket): usually no move or one step, else a seek.
+__device__ __forceinline__ int step_down(int k, int d, const int* edges, float log2_ex,
+                                         float log_scale) {
+  if (k == 0 || edges[k] <= d) return k;
+  if (edges[k - 1] <= d) return k - 1;
+  return seek_bucket(k - 1, d, edges, log2_ex, log_scale);
+}
+
 // Decides, for tile ti, the loaded pages and whether the relative-row chunk
 // [c0, c0+ROWS) must move so that it covers every bucket the tile needs.
 // All roles call it with identical arguments, so they agree on the sequence.
 template <int ROWS>
-__device__ __forceinline__ TilePlan plan_tile(const SplitGeom& g, int ti, int ex, const int* edges,
-                                              PlanState& st) {
+__device__ __forceinline__ TilePlan plan_tile(const SplitGeom& g, int ti, int ex, float log2_ex,
+                                              float log_scale, const int* edges, PlanState& st) {
   TilePlan t;
   const int pg = g.sp_begin + 2 * ti;
   t.j0 = pg * kPage;
@@ -197,12 +217,12 @@ __device__ __forceinline__ TilePlan plan_tile(const SplitGeom& g, int ti, int ex
   int b_hi = d_hi, b_lo = d_lo;
   t.k_hi = -1;
   if (d_hi >= ex) {
-    st.k_hi = step_down(st.k_hi, d_hi, edges);
+    st.k_hi = step_down(st.k_hi, d_hi, edges, log2_ex, log_scale);
     t.k_hi = st.k_hi;
     b_hi = ex + st.k_hi;
   }
   if (d_lo >= ex) {
-    st.k_lo = step_down(st.k_lo, d_lo, edges);
+    st.k_lo = step_down(st.k_lo, d_lo, edges, log2_ex, log_scale);
     b_lo = ex + st.k_lo;
   }
   t.chunk = !(st.have && b_lo >= st.c0 && b_hi < st.c0 + ROWS);
@@ -406,7 +426,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           bt_next = bt_load((ti >> 4) + 1);
         }
         const bool odd = (NG == 2) && (ti & 1);
-        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.edges, odd ? ps1 : ps0);
+        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, p.edges, odd ? ps1 : ps0);
         const int c0 = odd ? ps1.c0 : ps0.c0;
         if (tp.chunk) {
           ok = __all_sync(0xffffffffu,
@@ -510,7 +530,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       };
       for (int ti = 0; ti < g.ntiles; ++ti) {
         const int gq = (NG == 2) ? (ti & 1) : 0;
-        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, gq ? ps1 : ps0);
+        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
         // P.V of the previous tile frees a V slot: issue it first unless this
         // tile's K data has already landed (then S first, so softmax starts).
         bool pv_pending = i > 0;
@@ -620,7 +640,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     RELATTN_TRACE(5, 63);
     for (int ti = 0; ti < g.ntiles; ++ti) {
       const int owner = (NG == 2) ? (ti & 1) : 0;
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, s_edges, owner ? ps1 : ps0);
+      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, owner ? ps1 : ps0);
       const int c0 = owner ? ps1.c0 : ps0.c0;
       if (tp.chunk) {
         if (owner == grp) {
@@ -688,7 +708,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             int k = tp.k_hi - (int)(e_hi[0] > d) - (int)(e_hi[1] > d) - (int)(e_hi[2] > d) -
                     (int)(e_hi[3] > d);
             k = max(k, 0);
-            if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges);
+            if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges, p.log2_ex, p.log_scale);
             bk = p.ex + k;
           }
           const int r = v ? bk - c0 : 0;

@@ -52,13 +52,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait until the phase with the given parity has completed.  Returns false
-// if the CTA-wide abort flag is raised or `limit_ns` elapses (then the flag
-// is raised here).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag,
-                                          uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Polling loop of mbar_wait, out of line: every wait site then costs one
+// test inline, and the loop's code exists once.
+__device__ __noinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity,
+                                            volatile int* abort_flag,
+                                            uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -68,6 +66,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
       return false;
     }
   }
+}
+
+// Wait until the phase with the given parity has completed.  Returns false
+// if the CTA-wide abort flag is raised or `limit_ns` elapses (then the flag
+// is raised here).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_poll(bar, parity, abort_flag, limit_ns);
 }
 
 // ------------------------------------------------------------------ fences
