@@ -199,6 +199,41 @@ __device__ __forceinline__ int step_down(int k, int d, const int* edges, float l
   return seek_bucket(k - 1, d, edges, log2_ex, log_scale);
 }
 
+// Pages [*begin, *end) of split s among S over the pages [first, last] a
+// sequence's queries can see.  Splits are balanced by cost, not by page
+// count: a page near the queries costs more than a far one (inside the
+// exact-distance range every tile needs its own relative-row chunk, and up
+// to a few thousand keys out the tail buckets are narrow), so the page at
+// distance rank q from the query end is weighted 8 + kCostExact [q < QE] +
+// kCostNear [q < QN] eighths.  The cumulative cost from the query end is
+// piecewise linear and is inverted per boundary; interior boundaries are
+// rounded to an even page offset so that tiles stay two pages long.
+constexpr int kCostExact = 5, kCostNear = 1;
+__host__ __device__ __forceinline__ void split_pages(int first, int last, int S, int s, int ex,
+                                                     int* begin, int* end) {
+  const int n = last - first + 1;
+  const int qe = min(n, (ex + 128 + kPage - 1) / kPage + 1);   // pages holding exact-range keys
+  const int qn = min(n, max(qe, 8 * ex / kPage));              // pages of the narrow tail buckets
+  constexpr int s1 = 8 + kCostExact + kCostNear, s2 = 8 + kCostNear;
+  const int ce = s1 * qe;                                      // cost of the first qe pages
+  const int cn = ce + s2 * (qn - qe);                          // ... of the first qn pages
+  const int total = cn + 8 * (n - qn);                         // < 2^31 for n < 2^27 pages
+  const int tq = total / S, tr = total % S;
+  auto boundary = [&](int j) -> int {                           // page index of boundary j
+    if (j <= 0) return last + 1;
+    if (j >= S) return first;
+    const int c = tq * j + tr * j / S;                         // floor(total * j / S)
+    int q;
+    if (c <= ce) q = (c + s1 - 1) / s1;
+    else if (c <= cn) q = qe + (c - ce + s2 - 1) / s2;
+    else q = qn + (c - cn + 7) / 8;
+    const int b = last + 1 - min(q, n);
+    return first + ((b - first) & ~1);
+  };
+  *begin = boundary(S - s);
+  *end = boundary(S - 1 - s);
+}
+
 // Decides, for tile ti, the loaded pages and whether the relative-row chunk
 // [c0, c0+ROWS) must move so that it covers every bucket the tile needs.
 // All roles call it with identical arguments, so they agree on the sequence.
@@ -300,15 +335,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   g.p0 = g.L - T;
   g.W = p.window;
   g.lo = (g.W > 0) ? max(0, g.p0 - g.W + 1) : 0;
-  {
-    const int first = g.lo / kPage, last = (g.L - 1) / kPage;
-    const int n_pages = last - first + 1;
-    const int S = p.num_splits;
-    const int pps = 2 * ((n_pages + 2 * S - 1) / (2 * S));
-    g.sp_begin = first + s_idx * pps;
-    g.sp_end = min(g.sp_begin + pps, last + 1);
-    g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
-  }
+  split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, &g.sp_begin, &g.sp_end);
+  g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {                       // a trailing split with no page
     fill_rows<G>(p, b, h, s_idx, 0.f, -INFINITY);
     return;

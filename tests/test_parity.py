@@ -105,6 +105,17 @@ def test_bf16_output_is_rounded_fp32(ra):
         assert torch.equal(l32, l16)
 
 
+def test_split_count_invariance_long(ra):
+    """Splits are cost-weighted toward the query end: with 313 pages every
+    segment of the weighting (exact range, narrow tail buckets, far pages)
+    falls inside some split for these counts."""
+    case = small(20000, T=1)
+    ref = run_oracle(case)
+    for s in (2, 3, 5, 8, 13, 18, 37, 64, 150, 157):
+        out, lse = run_gpu(ra, case, s)
+        check(out, lse, *ref)
+
+
 def test_split_count_invariance_small(ra):
     case = small(5000, T=1)
     ref = run_oracle(case)
