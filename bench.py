@@ -205,6 +205,27 @@ def torch_arange_row(n):
     return torch.arange(n, dtype=torch.int32)[None]
 
 
+# ------------------------------------------------------- multi-rank timing
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's device time: every rank contributes its own total and
+    all receive the maximum (the process group's backend: NCCL on GPUs, gloo
+    in the CPU tests)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, steps: int, bytes_per_step: int, total_ms: float) -> float:
+    """Aggregate throughput: every rank moves `bytes_per_step` per step (weak
+    scaling, one independent decode problem per rank), over the slowest
+    rank's time."""
+    return world * steps * bytes_per_step / (total_ms * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -260,11 +281,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     t_step = [e[0].elapsed_time(e[1]) for e in ev]
-    total_ms = sum(t_step)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(t_step), world, dev)
     status = prep.workspace.read_status()
 
     # Per-kernel durations: the same step with an event between the partial
@@ -313,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
         mean_step = total_ms / K
         mean_part = statistics.fmean(t_part)
         achieved = nbytes / (mean_part * 1e-3) / 1e9
-        value = world * K * nbytes / (total_ms * 1e-3) / 1e9
+        value = whole_job_gbs(world, K, nbytes, total_ms)
         src_hash = kernel_source_hash()
         cpu = None
         if not args.no_cpu_baseline and world == 1:
