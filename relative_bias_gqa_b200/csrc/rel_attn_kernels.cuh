@@ -98,7 +98,14 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 // ring (a V slot is held until the P.V product of its tile).
 template <int N, int NG>
 struct KernelConfig {
+  // N = 16 (one token): the softmax groups alternate tiles, each with all the
+  // rows.  N = 32 / 48 (2..8 tokens): both groups take every tile, each with
+  // its own block of rows (a column split of S^T, X^T and O^T).
+  static constexpr bool kAlt = (N == 16);
   static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
+  static constexpr int kConsumers = kAlt ? kSoftmaxThreads : kSoftmaxThreads * NG;  // arrivals per tile
+  static constexpr int kXTables = kAlt ? NG : 1;               // relative chunks in flight (X, Y)
+  static constexpr int kGR = kAlt ? N : N / 2;                 // row capacity of a group
   // relative rows per chunk: 128 cover one 128-key tile for one token; with
   // T tokens a tile needs 127 + T rows
   static constexpr int kRows = (N == 16) ? 128 : 136;
@@ -117,28 +124,27 @@ struct KernelConfig {
   static constexpr int oV = kKSlots * kKSlotBytes;
   static constexpr int oQ = oV + kVSlots * kVSlotBytes;
   static constexpr int oP = oQ + kOperandBytes;                // two P buffers
-  static constexpr int oY = oP + 2 * kPBufBytes;               // one table per group
-  static constexpr int oRed = oY + NG * kYBytes;               // [NG][2][4][N]
-  static constexpr int oLred = oRed + NG * 2 * 4 * N * 4;      // [NG][4][N]
-  static constexpr int oAlpha = oLred + NG * 4 * N * 4;        // [NG][2][N]
-  static constexpr int oEdges = oAlpha + NG * 2 * N * 4;
+  static constexpr int oY = oP + 2 * kPBufBytes;               // one table per relative chunk in flight
+  static constexpr int oRed = oY + kXTables * kYBytes;         // [NG][2][4][kGR]
+  static constexpr int oAlpha = oRed + NG * 2 * 4 * kGR * 4;   // [NG][2][kGR]
+  static constexpr int oEdges = oAlpha + NG * 2 * kGR * 4;
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
   // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s_full[2],
-  //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[NG],
-  //           x_empty[NG], drain
-  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 11 + 2 * NG;
+  //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[kXTables],
+  //           x_empty[kXTables], drain
+  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 11 + 2 * kXTables;
   static constexpr int oMisc = oBar + kNumBars * 8;            // tmem base, abort flag
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAllocBytes = kBytes + 1024;            // 1024-byte alignment slack
   // TMEM columns: S[2] (N each), O[2] (2N each: the P_hi and P_lo halves),
   // per group X0 (and X1 for 136-row chunks)
   static constexpr int kXCols = (kRows > 128) ? 2 * N : N;
-  static constexpr int kTmemUsed = 6 * N + kXCols * NG;
+  static constexpr int kTmemUsed = 6 * N + kXCols * kXTables;
   static constexpr int kTmemCols = (kTmemUsed <= 128) ? 128 : (kTmemUsed <= 256 ? 256 : 512);
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
   static_assert(kKSlotBytes >= 2 * kHalfTileBytes && oV % 1024 == 0 && oQ % 1024 == 0,
                 "slot layout");
-  static_assert(oV >= NG * N * 128 * 4 * 2 + NG * N * 4 * 2, "epilogue exchange area");
+  static_assert(oV >= NG * kGR * 128 * 4 * 2 + NG * kGR * 4 * 2, "epilogue exchange area");
 };
 
 // Per-CTA geometry shared by the three roles.
@@ -320,7 +326,18 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const int warp = tid >> 5, lane = tid & 31;
   const int s_idx = RELATTN_SPLIT_OF_BLOCK(blockIdx.x), h = RELATTN_HEAD_OF_BLOCK(blockIdx.y), b = blockIdx.z;
   constexpr int NQ = T * G;
-  static_assert(NQ <= N, "group width");
+  // rows per softmax group: all NQ when the groups alternate tiles; else
+  // group 0 takes the first TA tokens and group 1 the other TB, group 1's
+  // rows starting at query slot kSlot1 (8-aligned, so no 8-row block of P is
+  // shared by the groups)
+  constexpr int TA = KC::kAlt ? T : (T + 1) / 2;
+  constexpr int TB = KC::kAlt ? T : T - TA;
+  constexpr int RG = TA * G;
+  constexpr int RG8 = (RG + 7) / 8;
+  constexpr int kSlot1 = KC::kAlt ? 0 : align_up(RG, 8);
+  constexpr bool kEvenSplit = KC::kAlt || TA == TB;
+  static_assert(NG == 2, "two softmax groups");
+  static_assert(KC::kAlt ? NQ <= N : (kSlot1 + TB * G <= N && RG <= KC::kGR), "group width");
   RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
@@ -359,8 +376,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t o_full = bar0 + 8u * (kB + 6);
   const uint32_t o_empty = bar0 + 8u * (kB + 8);
   const uint32_t x_full = bar0 + 8u * (kB + 10);   // +8*group
-  const uint32_t x_empty = bar0 + 8u * (kB + 10 + NG);
-  const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * NG);
+  const uint32_t x_empty = bar0 + 8u * (kB + 10 + KC::kXTables);
+  const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * KC::kXTables);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 4);
   auto kslot = [&](int k) { return sbase + KC::oK + (uint32_t)((k % KS) * KC::kKSlotBytes); };
@@ -381,14 +398,14 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(s_full + 8u * i, 1);
-      ptx::mbar_init(s_empty + 8u * i, kSoftmaxThreads);
-      ptx::mbar_init(p_full + 8u * i, kSoftmaxThreads);
+      ptx::mbar_init(s_empty + 8u * i, KC::kConsumers);
+      ptx::mbar_init(p_full + 8u * i, KC::kConsumers);
       ptx::mbar_init(o_full + 8u * i, 1);
-      ptx::mbar_init(o_empty + 8u * i, kSoftmaxThreads);
+      ptx::mbar_init(o_empty + 8u * i, KC::kConsumers);
     }
-    for (int gq = 0; gq < NG; ++gq) {
+    for (int gq = 0; gq < KC::kXTables; ++gq) {
       ptx::mbar_init(x_full + 8u * gq, 1);
-      ptx::mbar_init(x_empty + 8u * gq, kSoftmaxThreads);
+      ptx::mbar_init(x_empty + 8u * gq, KC::kConsumers);
     }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -406,12 +423,16 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     } else {
       const int st = tid - 64;
       const int nst = kSoftmaxThreads * NG;
-      // Q group tile: rows n = t*G + g (padding rows zero), 128B-swizzled K-major.
+      // Q group tile, 128B-swizzled K-major: query slot n holds (token t,
+      // head gg) with n = t*G + gg, except that with column-split groups
+      // group 1's tokens start at slot kSlot1; other slots are zero.
       for (int u = st; u < N * 16; u += nst) {
         const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < NQ) {
-          const int t = n / G, gg = n % G;
+        const int nl = (n >= kSlot1 && !KC::kAlt) ? n - kSlot1 + TA * G : n;   // row t*G + gg
+        const bool used = KC::kAlt ? n < NQ : (n < kSlot1 ? n < RG : nl < NQ);
+        if (used) {
+          const int t = nl / G, gg = nl % G;
           const __nv_bfloat16* src = p.q + ((size_t)(b * T + t) * p.Hq + h * G + gg) * kHeadDim
                                      + half * 64 + w16 * 8;
           v = __ldg(reinterpret_cast<const uint4*>(src));
@@ -453,7 +474,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           bt_cur = bt_next;
           bt_next = bt_load((ti >> 4) + 1);
         }
-        const bool odd = (NG == 2) && (ti & 1);
+        const bool odd = KC::kAlt && (ti & 1);
         const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, p.edges, odd ? ps1 : ps0);
         const int c0 = odd ? ps1.c0 : ps0.c0;
         if (tp.chunk) {
@@ -557,7 +578,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         return true;
       };
       for (int ti = 0; ti < g.ntiles; ++ti) {
-        const int gq = (NG == 2) ? (ti & 1) : 0;
+        const int gq = KC::kAlt ? (ti & 1) : 0;
         const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
         // P.V of the previous tile frees a V slot: issue it first unless this
         // tile's K data has already landed (then S first, so softmax starts).
@@ -618,45 +639,51 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   }
   // --------------------------------------------------------------- softmax
   else {
-    const int grp = (NG == 2) ? (warp - 2) >> 2 : 0;   // softmax group of this warp
+    const int grp = (warp - 2) >> 2;          // softmax group of this warp
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
     const int kl = sp * 32 + lane;            // key lane (S^T) / head-dim lane (O^T)
     const int wsm = (warp - 2) & 3;           // warp index inside the group
     const int bar_id = 1 + grp;
     const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-    float* Y = reinterpret_cast<float*>(smem + KC::oY + grp * KC::kYBytes);
-    float* red = reinterpret_cast<float*>(smem + KC::oRed) + grp * 2 * 4 * N;
-    float* alpha_buf = reinterpret_cast<float*>(smem + KC::oAlpha) + grp * 2 * N;
-    const uint32_t tXg = tX(grp) + lane_off;
+    // this group's rows: query slots [slot0, slot0 + RG), tokens from tok0;
+    // `nrows` of them are live (fewer than RG only for group 1 at odd T)
+    const int slot0 = KC::kAlt ? 0 : grp * kSlot1;
+    const int tok0 = KC::kAlt ? 0 : grp * TA;
+    const int nrows = KC::kAlt ? NQ : (grp ? TB * G : TA * G);
+    auto live = [&](int r) { return r < RG && (kEvenSplit || r < nrows); };
+    float* Y = reinterpret_cast<float*>(smem + KC::oY + (KC::kAlt ? grp : 0) * KC::kYBytes);
+    float* red = reinterpret_cast<float*>(smem + KC::oRed) + grp * 2 * 4 * KC::kGR;
+    float* alpha_buf = reinterpret_cast<float*>(smem + KC::oAlpha) + grp * 2 * KC::kGR;
+    const uint32_t tXg = tX(KC::kAlt ? grp : 0) + lane_off + slot0;
     // per-row running state: l (this thread's keys), O (this thread's head-dim
     // lane), reference max; alpha_r carries this tile's rescale factors when
-    // O is taken right away (two groups)
-    float l_part[N], o_acc[N], m_ref[N];
-    float alpha_r[NG == 2 ? N : 1];
+    // O is taken right away (alternating groups)
+    float l_part[RG], o_acc[RG], m_ref[RG];
+    float alpha_r[KC::kAlt ? RG : 1];
 #pragma unroll
-    for (int n = 0; n < N; ++n) { l_part[n] = 0.f; o_acc[n] = 0.f; m_ref[n] = -INFINITY; }
+    for (int r = 0; r < RG; ++r) { l_part[r] = 0.f; o_acc[r] = 0.f; m_ref[r] = -INFINITY; }
 #pragma unroll
-    for (int n = 0; n < (NG == 2 ? N : 1); ++n) alpha_r[n] = 1.f;
+    for (int r = 0; r < (KC::kAlt ? RG : 1); ++r) alpha_r[r] = 1.f;
     int c = 0, li = 0;                        // own chunks, own tiles
     PlanState ps0(p.nl), ps1(p.nl);
     bool failed = false, aborted = false;
 
-    // Accumulate the O^T tile of tile j (this thread's head-dim lane) with
-    // the rescale factors `al` of that tile.
+    // Accumulate the O^T tile of tile j (this thread's head-dim lane, this
+    // group's columns) with the rescale factors `al` of that tile.
     auto process_o = [&](int j, const float* al) {
-      float ov[N];
+      float ov[RG8 * 8];
       const bool okw = ptx::mbar_wait(o_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N;
+        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N + slot0;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {          // O^T from P_hi, then from P_lo
 #pragma unroll
-          for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(ob + part * N + q16 * 16, ov + q16 * 16);
+          for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(ob + part * N + q8 * 8, ov + q8 * 8);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int n = 0; n < N; ++n)
-            if (n < NQ) o_acc[n] = part ? o_acc[n] + ov[n] : fmaf(o_acc[n], al[n], ov[n]);
+          for (int r = 0; r < RG; ++r)
+            if (live(r)) o_acc[r] = part ? o_acc[r] + ov[r] : fmaf(o_acc[r], al[r], ov[r]);
         }
         ptx::tc_fence_before();
       }
@@ -667,35 +694,38 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     int last_tile = -1;
     RELATTN_TRACE(5, 63);
     for (int ti = 0; ti < g.ntiles; ++ti) {
-      const int owner = (NG == 2) ? (ti & 1) : 0;
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, owner ? ps1 : ps0);
-      const int c0 = owner ? ps1.c0 : ps0.c0;
+      const int owner = KC::kAlt ? (ti & 1) : grp;
+      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges,
+                                          (KC::kAlt && owner) ? ps1 : ps0);
+      const int c0 = (KC::kAlt && owner) ? ps1.c0 : ps0.c0;
       if (tp.chunk) {
         if (owner == grp) {
-          // ---- new relative-row chunk: X^T (136 rows x N) -> gather table Y
-          const bool okw = ptx::mbar_wait(x_full + 8u * grp, c & 1, abort_flag, tlim);
+          // ---- new relative-row chunk: this group's columns of X^T (128 or
+          //      136 relative rows) -> gather table Y
+          const int xb = KC::kAlt ? grp : 0;
+          const bool okw = ptx::mbar_wait(x_full + 8u * xb, c & 1, abort_flag, tlim);
           if (okw) {
-            float xv[N];
+            float xv[RG8 * 8];
             ptx::tc_fence_after();
 #pragma unroll
-            for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tXg + q16 * 16, xv + q16 * 16);
+            for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(tXg + q8 * 8, xv + q8 * 8);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int n = 0; n < N; ++n)
-              if (n < NQ) Y[kl * YS + n] = xv[n];
+            for (int r = 0; r < RG; ++r)
+              if (live(r)) Y[kl * YS + slot0 + r] = xv[r];
             if (ROWS > 128 && sp == 3) {         // rows 128..135 come from lanes 120..127 of X1
 #pragma unroll
-              for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tXg + N + q16 * 16, xv + q16 * 16);
+              for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(tXg + N + q8 * 8, xv + q8 * 8);
               ptx::tmem_wait_ld();
               if (lane >= 24) {
 #pragma unroll
-                for (int n = 0; n < N; ++n)
-                  if (n < NQ) Y[(kl + 8) * YS + n] = xv[n];
+                for (int r = 0; r < RG; ++r)
+                  if (live(r)) Y[(kl + 8) * YS + slot0 + r] = xv[r];
               }
             }
             ptx::tc_fence_before();
           }
-          ptx::mbar_arrive(x_empty + 8u * grp);
+          ptx::mbar_arrive(x_empty + 8u * xb);
           if (c == 0) RELATTN_TRACE(6, 63);
           ++c;
           if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
@@ -704,14 +734,15 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if (owner != grp) continue;
       const int i = ti;                       // buffers and phases follow the tile index
 
-      // ---- S^T tile: this thread owns key j
-      float s[N];
+      // ---- S^T tile: this thread owns key j, this group's columns
+      float s[RG8 * 8];
       const bool okw = ptx::mbar_wait(s_full + 8u * (i & 1), (i >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
         RELATTN_TRACE(4, i);
 #pragma unroll
-        for (int q16 = 0; q16 < N / 16; ++q16) ptx::tmem_ld16(tS + lane_off + (i & 1) * N + q16 * 16, s + q16 * 16);
+        for (int q8 = 0; q8 < RG8; ++q8)
+          ptx::tmem_ld8(tS + lane_off + (i & 1) * N + slot0 + q8 * 8, s + q8 * 8);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
       }
@@ -727,25 +758,23 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) e_hi[m] = s_edges[max(tp.k_hi - m, 0)];
 #pragma unroll
-      for (int t = 0; t < T; ++t) {
-        {
-          const int d = d0 + t;
-          const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
-          int bk = d;                               // exact region: the distance itself
-          if (v && d >= p.ex) {
-            int k = tp.k_hi - (int)(e_hi[0] > d) - (int)(e_hi[1] > d) - (int)(e_hi[2] > d) -
-                    (int)(e_hi[3] > d);
-            k = max(k, 0);
-            if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges, p.log2_ex, p.log_scale);
-            bk = p.ex + k;
-          }
-          const int r = v ? bk - c0 : 0;
-          const float* yrow = Y + r * YS;
+      for (int tt = 0; tt < TA; ++tt) {
+        if (!kEvenSplit && tt * G >= nrows) break;
+        const int d = d0 + tok0 + tt;
+        const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
+        int bk = d;                               // exact region: the distance itself
+        if (v && d >= p.ex) {
+          int k = tp.k_hi - (int)(e_hi[0] > d) - (int)(e_hi[1] > d) - (int)(e_hi[2] > d) -
+                  (int)(e_hi[3] > d);
+          k = max(k, 0);
+          if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges, p.log2_ex, p.log_scale);
+          bk = p.ex + k;
+        }
+        const float* yrow = Y + (v ? bk - c0 : 0) * YS + slot0;
 #pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            const int n = t * G + gg;
-            if (n < N) s[n] = v ? (s[n] + yrow[n]) * p.scale_log2 : -INFINITY;
-          }
+        for (int gg = 0; gg < G; ++gg) {
+          const int r = tt * G + gg;
+          s[r] = v ? (s[r] + yrow[r]) * p.scale_log2 : -INFINITY;
         }
       }
       // ---- lazy max: p = exp2(x - m_ref) with the row's reference max
@@ -755,37 +784,38 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       //      Results stay exact: lse = m_ref + log2(l) for any m_ref.
       bool over = false;
 #pragma unroll
-      for (int n = 0; n < N; ++n)
-        if (n < NQ) over |= s[n] > m_ref[n] + kLazyLog2;
-      float* al_buf = alpha_buf + (li & 1) * N;
+      for (int r = 0; r < RG; ++r)
+        if (live(r)) over |= s[r] > m_ref[r] + kLazyLog2;
+      float* al_buf = alpha_buf + (li & 1) * KC::kGR;
       if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, over || !okw || failed)) {
         if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
-        float* redb = red + (li & 1) * 4 * N;
+        float* redb = red + (li & 1) * 4 * KC::kGR;
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-          if (n < NQ) {
-            const float mx = warp_max(s[n]);
-            if (lane == 0) redb[wsm * N + n] = mx;
+        for (int r = 0; r < RG; ++r) {
+          if (live(r)) {
+            const float mx = warp_max(s[r]);
+            if (lane == 0) redb[wsm * KC::kGR + r] = mx;
           }
         }
         ptx::bar_sync_or(bar_id, kSoftmaxThreads, false);
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-          if (n < NQ) {
-            const float tmax = fmaxf(fmaxf(redb[n], redb[N + n]), fmaxf(redb[2 * N + n], redb[3 * N + n]));
-            const float mn = fmaxf(m_ref[n], tmax);
-            const float alpha = exp2f(m_ref[n] - ((mn == -INFINITY) ? 0.f : mn));
-            l_part[n] *= alpha;
-            if constexpr (NG == 2) alpha_r[n] = alpha;
-            else if (kl == 0) al_buf[n] = alpha;
-            m_ref[n] = mn;
+        for (int r = 0; r < RG; ++r) {
+          if (live(r)) {
+            const float tmax = fmaxf(fmaxf(redb[r], redb[KC::kGR + r]),
+                                     fmaxf(redb[2 * KC::kGR + r], redb[3 * KC::kGR + r]));
+            const float mn = fmaxf(m_ref[r], tmax);
+            const float alpha = exp2f(m_ref[r] - ((mn == -INFINITY) ? 0.f : mn));
+            l_part[r] *= alpha;
+            if constexpr (KC::kAlt) alpha_r[r] = alpha;
+            else if (kl == 0) al_buf[r] = alpha;
+            m_ref[r] = mn;
           }
         }
       } else {
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-          if constexpr (NG == 2) alpha_r[n] = 1.f;
-          else if (kl == 0 && n < NQ) al_buf[n] = 1.f;
+        for (int r = 0; r < RG; ++r) {
+          if constexpr (KC::kAlt) alpha_r[r] = 1.f;
+          else if (kl == 0 && live(r)) al_buf[r] = 1.f;
         }
       }
       RELATTN_TRACE(5, i);
@@ -793,21 +823,24 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       //      the P.V product), stacked [P_hi; P_lo] = 2N rows, MN-major without
       //      swizzle: 8-row x 16-byte core matrices, row blocks 128 B apart,
       //      8-key groups 32*N B apart; each thread writes its key with 16-byte
-      //      stores.
+      //      stores into the 8-row blocks of its group's slots (rows past the
+      //      group's live ones get zeros; slots no group owns are never read
+      //      back, as O^T column n depends on P row n only).
       {
         const uint32_t pbuf = sP0 + (uint32_t)((i & 1) * KC::kPBufBytes);
-        const uint32_t prow = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16);
+        const uint32_t prow = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16) +
+                              (uint32_t)(slot0 / 8) * 128;
 #pragma unroll
-        for (int cb = 0; cb < N / 8; ++cb) {
+        for (int cb = 0; cb < RG8; ++cb) {
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
-            const int n0 = cb * 8 + 2 * q2, n1 = n0 + 1;
+            const int r0 = cb * 8 + 2 * q2, r1 = r0 + 1;
             float p0 = 0.f, p1 = 0.f;
-            if (n0 < NQ) p0 = exp2f(s[n0] - ((m_ref[n0] == -INFINITY) ? 0.f : m_ref[n0]));
-            if (n1 < NQ) p1 = exp2f(s[n1] - ((m_ref[n1] == -INFINITY) ? 0.f : m_ref[n1]));
-            if (n0 < NQ) l_part[n0] += p0;
-            if (n1 < NQ) l_part[n1] += p1;
+            if (live(r0)) p0 = exp2f(s[r0] - ((m_ref[r0] == -INFINITY) ? 0.f : m_ref[r0]));
+            if (live(r1)) p1 = exp2f(s[r1] - ((m_ref[r1] == -INFINITY) ? 0.f : m_ref[r1]));
+            if (live(r0)) l_part[r0] += p0;
+            if (live(r1)) l_part[r1] += p1;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - __low2float(h2), p1 - __high2float(h2));
             hi[q2] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -821,8 +854,9 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
       }
       // ---- keys no token may see: clear their V rows (stale or poisoned data
-      //      must not reach the P.V product, where 0 * NaN = NaN)
-      {
+      //      must not reach the P.V product, where 0 * NaN = NaN); with both
+      //      groups on the tile, group 0 does it
+      if (KC::kAlt || grp == 0) {
         const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
         if (!any_valid) {
           volatile int never = 0;
@@ -838,74 +872,84 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
       RELATTN_TRACE(6, i);
-      if constexpr (NG == 2) {
+      if constexpr (KC::kAlt) {
         // this group's next tile is i + 2: take O(i) now
         process_o(i, alpha_r);
         RELATTN_TRACE(7, i);
       } else {
+        // both groups are on every tile: take O(i-1) while P.V(i) runs
         if (last_tile >= 0) {
-          process_o(last_tile, alpha_buf + ((li - 1) & 1) * N);
+          process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
           RELATTN_TRACE(7, last_tile);
         }
       }
       last_tile = i;
       ++li;
     }
-    if constexpr (NG == 1) {
+    if constexpr (!KC::kAlt) {
       if (!aborted) {
         if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, failed)) aborted = true;
-        else if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * N);
+        else if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
       }
     }
     ptx::pdl_launch_dependents();
 
     // ---- epilogue: each group's unnormalised O, per-lane l and reference
     //      max go to shared memory (the K ring, idle once every S has been
-    //      read); then all softmax threads merge the groups and write this
-    //      CTA's rows in short loops.
+    //      read); then all softmax threads finish the rows in short loops.
+    //      Alternating groups hold the same rows (merged by LSE); column-split
+    //      groups hold disjoint rows.
     bool bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, aborted || failed);
-    float* eo = reinterpret_cast<float*>(smem);             // [NG][NQ][128]
-    float* el = eo + NG * NQ * kHeadDim;                    // [NG][NQ][128]
-    float* em = el + NG * NQ * kHeadDim;                    // [NG][NQ]
-    float* es = em + NG * NQ;                               // [NG][NQ]
+    float* eo = reinterpret_cast<float*>(smem);             // [NG][RG][128]
+    float* el = eo + NG * RG * kHeadDim;                    // [NG][RG][128]
+    float* em = el + NG * RG * kHeadDim;                    // [NG][RG]
+    float* es = em + NG * RG;                               // [NG][RG]
     if (!bad) {
 #pragma unroll
-      for (int n = 0; n < NQ; ++n) {
-        eo[(grp * NQ + n) * kHeadDim + kl] = o_acc[n];
-        el[(grp * NQ + n) * kHeadDim + kl] = l_part[n];
+      for (int r = 0; r < RG; ++r) {
+        eo[(grp * RG + r) * kHeadDim + kl] = o_acc[r];
+        el[(grp * RG + r) * kHeadDim + kl] = l_part[r];
       }
       if (kl == 0) {
 #pragma unroll
-        for (int n = 0; n < NQ; ++n) em[grp * NQ + n] = m_ref[n];
+        for (int r = 0; r < RG; ++r) em[grp * RG + r] = m_ref[r];
       }
     }
     bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, bad);
     if (!bad) {
       const int et = tid - 64, ew = et >> 5;               // softmax thread / warp index
       // row sums of l: one warp per (group, row)
-      for (int r = ew; r < NG * NQ; r += 4 * NG) {
-        const float* src = el + r * kHeadDim;
+      for (int q = ew; q < NG * RG; q += 4 * NG) {
+        const float* src = el + q * kHeadDim;
         const float v = warp_sum(src[lane] + src[lane + 32] + src[lane + 64] + src[lane + 96]);
-        if (lane == 0) es[r] = v;
+        if (lane == 0) es[q] = v;
       }
       ptx::bar_sync_or(3, kSoftmaxThreads * NG, false);
       const int rows = p.B * T * p.Hq;
+      // output rows: (token t, head gg) <- entries (group, local row)
       for (int e = et; e < NQ * kHeadDim; e += kSoftmaxThreads * NG) {
         const int n = e / kHeadDim, d = e % kHeadDim;
-        float m = -INFINITY;
+        const int t = n / G, gg = n - t * G;
+        float m = -INFINITY, o = 0.f, l = 0.f;
+        if constexpr (KC::kAlt) {
 #pragma unroll
-        for (int q = 0; q < NG; ++q) m = fmaxf(m, em[q * NQ + n]);
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float o = 0.f, l = 0.f;
+          for (int q = 0; q < NG; ++q) m = fmaxf(m, em[q * RG + n]);
+          const float mu = (m == -INFINITY) ? 0.f : m;
 #pragma unroll
-        for (int q = 0; q < NG; ++q) {
-          const float sc = exp2f(em[q * NQ + n] - mu);
-          o = fmaf(eo[(q * NQ + n) * kHeadDim + d], sc, o);
-          l = fmaf(es[q * NQ + n], sc, l);
+          for (int q = 0; q < NG; ++q) {
+            const float sc = exp2f(em[q * RG + n] - mu);
+            o = fmaf(eo[(q * RG + n) * kHeadDim + d], sc, o);
+            l = fmaf(es[q * RG + n], sc, l);
+          }
+        } else {
+          const int q = (t >= TA) ? 1 : 0;
+          const int idx = q * RG + (t - q * TA) * G + gg;
+          m = em[idx];
+          o = eo[idx * kHeadDim + d];
+          l = es[idx];
         }
         o = (l > 0.f) ? o / l : 0.f;
         const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int t = n / G, gg = n - t * G;
         const int row = (b * T + t) * p.Hq + h * G + gg;
         if (p.num_splits == 1) {
           if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
