@@ -67,6 +67,10 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s
 // Lazy-max slack (log2 units): p = exp2(x - m_ref) may reach 2^64, far
 // inside fp32 / bf16 range even summed over 2^31 keys.
 constexpr float kLazyLog2 = 64.f;
+// Reference max of a row before its first valid logit: finite, so that
+// exp2(x - m) and exp2(m_old - m_new) need no special case (any finite
+// logit exceeds it by more than kLazyLog2 and sets a real reference).
+constexpr float kNoMax = -1.0e30f;
 
 struct alignas(64) DecodeParams {
   CUtensorMap tmap_k;   // K pool viewed as [num_pages*Hkv*P rows, 128] bf16
@@ -194,6 +198,13 @@ __device__ __forceinline__ int seek_bucket(int k, int d, const int* edges, float
     if (edges[mid] <= d) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// Out-of-line seek for the rare key whose bucket lies more than a few
+// below its tile's largest (keeps the unrolled per-token code small).
+__device__ __noinline__ int seek_bucket_far(int k, int d, const int* edges, float log2_ex,
+                                            float log_scale) {
+  return seek_bucket(k, d, edges, log2_ex, log_scale);
 }
 
 // Moves cursor k down to the tail bucket of d (d never lies above the
@@ -661,7 +672,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     float l_part[RG], o_acc[RG], m_ref[RG];
     float alpha_r[KC::kAlt ? RG : 1];
 #pragma unroll
-    for (int r = 0; r < RG; ++r) { l_part[r] = 0.f; o_acc[r] = 0.f; m_ref[r] = -INFINITY; }
+    for (int r = 0; r < RG; ++r) { l_part[r] = 0.f; o_acc[r] = 0.f; m_ref[r] = kNoMax; }
 #pragma unroll
     for (int r = 0; r < (KC::kAlt ? RG : 1); ++r) alpha_r[r] = 1.f;
     int c = 0, li = 0;                        // own chunks, own tiles
@@ -767,7 +778,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           int k = tp.k_hi - (int)(e_hi[0] > d) - (int)(e_hi[1] > d) - (int)(e_hi[2] > d) -
                   (int)(e_hi[3] > d);
           k = max(k, 0);
-          if (k > 0 && s_edges[k] > d) k = step_down(k, d, s_edges, p.log2_ex, p.log_scale);
+          if (k > 0 && s_edges[k] > d) k = seek_bucket_far(k, d, s_edges, p.log2_ex, p.log_scale);
           bk = p.ex + k;
         }
         const float* yrow = Y + (v ? bk - c0 : 0) * YS + slot0;
@@ -804,7 +815,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             const float tmax = fmaxf(fmaxf(redb[r], redb[KC::kGR + r]),
                                      fmaxf(redb[2 * KC::kGR + r], redb[3 * KC::kGR + r]));
             const float mn = fmaxf(m_ref[r], tmax);
-            const float alpha = exp2f(m_ref[r] - ((mn == -INFINITY) ? 0.f : mn));
+            const float alpha = exp2f(m_ref[r] - mn);
             l_part[r] *= alpha;
             if constexpr (KC::kAlt) alpha_r[r] = alpha;
             else if (kl == 0) al_buf[r] = alpha;
@@ -837,8 +848,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           for (int q2 = 0; q2 < 4; ++q2) {
             const int r0 = cb * 8 + 2 * q2, r1 = r0 + 1;
             float p0 = 0.f, p1 = 0.f;
-            if (live(r0)) p0 = exp2f(s[r0] - ((m_ref[r0] == -INFINITY) ? 0.f : m_ref[r0]));
-            if (live(r1)) p1 = exp2f(s[r1] - ((m_ref[r1] == -INFINITY) ? 0.f : m_ref[r1]));
+            if (live(r0)) p0 = exp2f(s[r0] - m_ref[r0]);
+            if (live(r1)) p1 = exp2f(s[r1] - m_ref[r1]);
             if (live(r0)) l_part[r0] += p0;
             if (live(r1)) l_part[r1] += p1;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
