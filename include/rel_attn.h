@@ -183,6 +183,17 @@ int rel_attn_choose_splits(const rel_attn_shape* shape, int window, int sm_count
  * edge table), for tests.  Returns -1 for an invalid shape or distance < 0. */
 int rel_attn_bucket(const rel_attn_shape* shape, int distance);
 
+/* The pages [*first_page, *end_page) of a sequence of `seq_len` keys (its
+ * q_tokens queries at the end) that split `split` of `num_splits` walks:
+ * the same cost-weighted partition the partial kernel computes on the
+ * device (pages holding keys inside the exact-distance range weigh more
+ * than far pages; interior boundaries fall on even page offsets).  For
+ * tests and inspection; nothing is launched.  Returns 0, or
+ * REL_ATTN_ERR_INVALID_ARG for an invalid shape, seq_len < q_tokens or
+ * beyond the block-table row, or split outside [0, num_splits). */
+int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                         int split, int* first_page, int* end_page);
+
 /* Static description of an error code. */
 const char* rel_attn_error_string(int code);
 

@@ -18,6 +18,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxQTokens = 8;         // query tokens per sequence (speculative verify)
+constexpr int kMaxSplits = 256;
 constexpr size_t kHeaderBytes = 256;   // status word lives here
 
 struct DeviceInfo {
@@ -311,6 +312,22 @@ int rel_attn_bucket(const rel_attn_shape* shape, int distance) {
   static thread_local int edges[kMaxTailBuckets + 1];
   bucket_table_cached(shape, &ex, &nl, edges);
   return bucket_host(distance, ex, nl, edges);
+}
+
+int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                         int split, int* first_page, int* end_page) {
+  if (validate_shape(shape) != REL_ATTN_OK || !first_page || !end_page) return REL_ATTN_ERR_INVALID_ARG;
+  if (seq_len < shape->q_tokens || seq_len > shape->max_pages_per_seq * kPage)
+    return REL_ATTN_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > kMaxSplits || split < 0 || split >= num_splits)
+    return REL_ATTN_ERR_INVALID_ARG;
+  int ex, nl;
+  static thread_local int edges[kMaxTailBuckets + 1];
+  bucket_table_cached(shape, &ex, &nl, edges);
+  const int p0 = seq_len - shape->q_tokens;
+  const int lo = (window > 0) ? std::max(0, p0 - window + 1) : 0;
+  split_pages(lo / kPage, (seq_len - 1) / kPage, num_splits, split, ex, first_page, end_page);
+  return REL_ATTN_OK;
 }
 
 int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {

@@ -245,7 +245,7 @@ __host__ __device__ __forceinline__ void split_pages(int first, int last, int S,
     else if (c <= cn) q = qe + (c - ce + s2 - 1) / s2;
     else q = qn + (c - cn + 7) / 8;
     const int b = last + 1 - min(q, n);
-    return first + ((b - first) & ~1);
+    return min(first + ((b - first + 1) & ~1), last + 1); // nearest even offset, ties toward the query
   };
   *begin = boundary(S - s);
   *end = boundary(S - 1 - s);

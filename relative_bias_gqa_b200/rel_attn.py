@@ -27,6 +27,7 @@ EXPORTED = (
     "rel_attn_decode", "rel_attn_partial", "rel_attn_combine", "rel_attn_workspace_bytes", "rel_attn_workspace_init",
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
+    "rel_attn_split_pages",
 )
 
 
@@ -69,6 +70,9 @@ def _load():
     lib.rel_attn_choose_splits.restype = ctypes.c_int
     lib.rel_attn_bucket.argtypes = [SP, ctypes.c_int]
     lib.rel_attn_bucket.restype = ctypes.c_int
+    lib.rel_attn_split_pages.argtypes = [SP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.rel_attn_split_pages.restype = ctypes.c_int
     lib.rel_attn_error_string.argtypes = [ctypes.c_int]
     lib.rel_attn_error_string.restype = ctypes.c_char_p
     lib.rel_attn_version.argtypes = []
@@ -120,6 +124,17 @@ def rel_attn_choose_splits(shape: RelAttnShape, window: int, sm_count: int = 0) 
 
 def rel_attn_bucket(shape: RelAttnShape, distance: int) -> int:
     return int(lib.rel_attn_bucket(ctypes.byref(shape), int(distance)))
+
+
+def rel_attn_split_pages(shape: RelAttnShape, seq_len: int, window: int, num_splits: int,
+                         split: int):
+    """(first_page, end_page) of one split, as the partial kernel walks it."""
+    a, b = ctypes.c_int(), ctypes.c_int()
+    rc = lib.rel_attn_split_pages(ctypes.byref(shape), int(seq_len), int(window), int(num_splits),
+                                  int(split), ctypes.byref(a), ctypes.byref(b))
+    if rc != REL_ATTN_OK:
+        raise RelAttnError(rc)
+    return a.value, b.value
 
 
 def _stream_ptr(stream) -> int:

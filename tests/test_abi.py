@@ -136,3 +136,42 @@ def test_no_device_reported_without_gpu(ra):
 def test_error_strings(ra):
     for code in range(-6, 1):
         assert ra.error_string(code) and ra.error_string(code) != "unknown error"
+
+
+@pytest.mark.parametrize("L,T,window,nb", [(100_000, 1, 0, 1280), (262_144, 8, 0, 1280),
+                                            (100_000, 1, 1024, 1024), (20_000, 3, 0, 1280),
+                                            (5, 1, 0, 1280), (2048, 2, 100, 364)])
+def test_split_pages_partition(ra, L, T, window, nb):
+    """Every split count gives contiguous, ordered page ranges that cover
+    exactly the pages some query can see, tiles stay two pages long inside,
+    and near-query splits are no longer than far ones."""
+    pages = (L + 63) // 64 + 1
+    s = shape(ra, q_tokens=T, num_buckets=nb, max_pages_per_seq=pages, num_pages=pages,
+              max_seq_len=L, exact_buckets=min(1024, nb) if nb <= 1024 else 1024)
+    lo = max(0, L - T - window + 1) if window > 0 else 0
+    first, last = lo // 64, (L - 1) // 64
+    for S in (1, 2, 3, 7, 18, 37, 64, 148, 256):
+        prev = first
+        sizes = []
+        for sp in range(S):
+            a, b = ra.rel_attn_split_pages(s, L, window, S, sp)
+            assert a == prev and b >= a
+            assert (a - first) % 2 == 0 or a == last + 1      # inner boundaries keep 2-page tiles
+            sizes.append(b - a)
+            prev = b
+        assert prev == last + 1
+        big = [x for x in sizes if x > 0]
+        if len(big) > 2:
+            assert big[-1] <= max(big[:-1])
+
+
+def test_split_pages_rejects_bad_arguments(ra):
+    s = shape(ra)
+    import ctypes
+    a, b = ctypes.c_int(), ctypes.c_int()
+    f = ra.lib.rel_attn_split_pages
+    assert f(ctypes.byref(s), 100, 0, 4, 4, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), 100, 0, 0, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), 0, 0, 4, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), 1 << 30, 0, 4, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), 100, 0, 4, 0, None, ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
