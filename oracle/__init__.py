@@ -19,4 +19,7 @@ from .rel_attn_ref import (  # noqa: F401
     rel_attn_decode_ref,
     rel_attn_decode_split_ref,
     rel_attn_decode_bruteforce,
+    e4m3_to_float,
+    dequant_kv,
+    rel_attn_decode_fp8kv_ref,
 )

@@ -330,3 +330,52 @@ def rel_attn_decode_bruteforce(q, k_cache, v_cache, block_table, seq_lens,
                     out[b][t][hq][c] = sum(math.exp(x - lse_v) * v[c]
                                            for x, v in zip(logits, vals))
     return np.asarray(out), np.asarray(lse)
+
+
+# --------------------------------------------------------------------------
+# FP8 (e4m3) KV cache
+# --------------------------------------------------------------------------
+# "vLLM TML Inkling 지원", section "미래 로드맵", plans FP8 for the global
+# (full-context) attention layers to cut the KV-cache bottleneck; the
+# Reflection Beam page's serving example runs an FP8 KV cache.  Neither fixes
+# the format or the scales.  Reading taken: the OFP8 E4M3 format (1 sign bit,
+# 4 exponent bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 is
+# NaN) and one fp32 scale per KV head for K and one for V:
+#     k_j = e4m3(k_code_j) * k_scale[h],   v_j = e4m3(v_code_j) * v_scale[h].
+def e4m3_to_float(codes) -> np.ndarray:
+    """Real value of each E4M3 byte code, from the bit fields."""
+    c = np.asarray(codes).astype(np.int64) & 0xFF
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    exp = (c >> 3) & 0xF
+    man = (c & 0x7).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + man / 8.0, (exp - 7).astype(np.int64))
+    subnormal = sign * np.ldexp(man / 8.0, -6)
+    v = np.where(exp == 0, subnormal, normal)
+    return np.where((c & 0x7F) == 0x7F, np.nan, v)
+
+
+def dequant_kv(codes, scale) -> np.ndarray:
+    """[num_pages, Hkv, P, D] byte codes times the per-KV-head scale."""
+    v = e4m3_to_float(np.asarray(codes))
+    sc = np.asarray(_as_np(scale), dtype=np.float64).reshape(1, -1, 1, 1)
+    return v * sc
+
+
+def rel_attn_decode_fp8kv_ref(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                              rel_table, window: int, exact_buckets: int = EXACT_BUCKETS,
+                              max_distance: int = MAX_DISTANCE, batch_indices=None):
+    """The operation over an E4M3 KV cache: dequantise exactly (fp64), then the
+    same definition as rel_attn_decode_ref.  k_codes / v_codes are uint8
+    [num_pages, Hkv, P, D] (numpy, or torch uint8 / float8_e4m3fn viewed as
+    uint8); k_scale / v_scale are [Hkv]."""
+    def codes_of(x):
+        if hasattr(x, "detach"):
+            x = x.detach().cpu()
+            if x.element_size() == 1 and x.dtype.is_floating_point:
+                x = x.view(__import__("torch").uint8)
+            return x.numpy()
+        return np.asarray(x)
+    k = dequant_kv(codes_of(k_codes), k_scale)
+    v = dequant_kv(codes_of(v_codes), v_scale)
+    return rel_attn_decode_ref(q, k, v, block_table, seq_lens, rel_table, window,
+                               exact_buckets, max_distance, batch_indices)

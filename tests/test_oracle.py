@@ -342,3 +342,95 @@ def test_planted_reversed_distance(monkeypatch):
         kp = np.asarray(kp)
         return good(q, qp, k[::-1], v[::-1], kp, *a, **kw)
     assert _pins_fail(monkeypatch, "attend_at_positions", bad) > 0
+
+
+# ------------------------------------------------------- FP8 (E4M3) KV cache
+def test_e4m3_known_codes():
+    """Values fixed by the E4M3 bit layout (bias 7, 3 mantissa bits)."""
+    v = oracle.e4m3_to_float(np.array([0x00, 0x80, 0x38, 0xB8, 0x7E, 0xFE, 0x01, 0x07, 0x08,
+                                       0x3C, 0x40, 0x7F, 0xFF]))
+    want = [0.0, -0.0, 1.0, -1.0, 448.0, -448.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6,
+            1.5, 2.0]
+    assert np.array_equal(v[:11], want)
+    assert math.copysign(1.0, v[1]) == -1.0
+    assert np.isnan(v[11]) and np.isnan(v[12])
+
+
+def test_e4m3_matches_library_decode():
+    """Every code against torch's float8_e4m3fn decoding."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    lib = codes.view(torch.float8_e4m3fn).double().numpy()
+    mine = oracle.e4m3_to_float(codes.numpy())
+    assert np.array_equal(np.isnan(mine), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    assert np.array_equal(mine[ok], lib[ok])
+
+
+def fp8_case(seed=0, L=37, T=1, window=0):
+    case = small_case(L=L, T=T, window=window, seed=seed)
+    g = np.random.default_rng(seed + 7)
+    shape = tuple(case.k_cache.shape)
+    codes = lambda: g.integers(0, 256, size=shape, dtype=np.uint8) & 0xF7 | 0x30  # exponent 6 or 14: finite
+    kc, vc = codes(), codes()
+    Hkv = shape[1]
+    ks = g.uniform(0.01, 0.05, Hkv)
+    vs = g.uniform(0.5, 2.0, Hkv)
+    return case, kc, vc, ks, vs
+
+
+def run_fp8(case, kc, vc, ks, vs):
+    return oracle.rel_attn_decode_fp8kv_ref(case.q, kc, vc, ks, vs, case.block_table,
+                                            case.seq_lens, case.rel_table, case.window,
+                                            exact_buckets=case.exact_buckets,
+                                            max_distance=case.max_distance)
+
+
+def test_fp8kv_is_the_bf16_definition_on_decoded_values():
+    """Dequantised by hand (code value x scale, built from the format's bit
+    fields in the brute-force style) and fed to the pure-Python brute force."""
+    case, kc, vc, ks, vs = fp8_case(seed=3, L=23, T=2)
+
+    def decode(x):
+        s = -1.0 if x & 0x80 else 1.0
+        e, m = (x >> 3) & 0xF, x & 7
+        return s * (m / 8.0) * 2.0 ** -6 if e == 0 else s * (1 + m / 8.0) * 2.0 ** (e - 7)
+
+    dec = np.vectorize(decode, otypes=[np.float64])
+    k = dec(kc) * ks.reshape(1, -1, 1, 1)
+    v = dec(vc) * vs.reshape(1, -1, 1, 1)
+    o1, l1 = run_fp8(case, kc, vc, ks, vs)
+    o2, l2 = oracle.rel_attn_decode_bruteforce(case.q, k, v, case.block_table, case.seq_lens,
+                                               case.rel_table, case.window,
+                                               exact_buckets=case.exact_buckets,
+                                               max_distance=case.max_distance)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_fp8kv_v_scale_is_linear():
+    case, kc, vc, ks, vs = fp8_case(seed=1)
+    o1, l1 = run_fp8(case, kc, vc, ks, vs)
+    o2, l2 = run_fp8(case, kc, vc, ks, vs * 3.0)
+    assert np.allclose(o2, 3.0 * o1, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_fp8kv_zero_k_scale_leaves_the_relative_term():
+    """k_scale = 0 removes q.k: the result equals the definition with K = 0."""
+    case, kc, vc, ks, vs = fp8_case(seed=2, L=41)
+    o1, l1 = run_fp8(case, kc, vc, np.zeros_like(ks), vs)
+    v = oracle.dequant_kv(vc, vs)
+    o2, l2 = oracle.rel_attn_decode_ref(case.q, np.zeros_like(v), v, case.block_table,
+                                        case.seq_lens, case.rel_table, case.window,
+                                        exact_buckets=case.exact_buckets,
+                                        max_distance=case.max_distance)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_planted_e4m3_bias(monkeypatch):
+    """An exponent bias of 8 instead of 7 must fail the known-code pin."""
+    good = ref.e4m3_to_float
+
+    def bad(codes):
+        return good(codes) * 0.5
+    monkeypatch.setattr(oracle, "e4m3_to_float", bad)
+    with pytest.raises(AssertionError):
+        test_e4m3_known_codes()
