@@ -130,6 +130,39 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
                      void* stream);
 
 /*
+ * rel_attn_decode_e4m3 / rel_attn_partial_e4m3 -- the same operation over an
+ * FP8 KV cache ("vLLM TML Inkling 지원", section "미래 로드맵", plans FP8 for
+ * the full-context layers to relieve the KV-cache bottleneck; the pages fix
+ * no format, so this library reads it as follows).
+ *
+ *   k_cache, v_cache  uint8 [num_pages, Hkv, 64, 128], OFP8 E4M3 codes
+ *                     (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ *                     0x7F / 0xFF are NaN), device memory, 16-byte aligned.
+ *   k_scale, v_scale  fp32 [Hkv], device memory, 4-byte aligned: key j of KV
+ *                     head h is e4m3(k_code) * k_scale[h], likewise for V.
+ * Every other argument, the workspace and the outputs are as for
+ * rel_attn_decode / rel_attn_partial (rel_attn_combine merges the splits of
+ * either).  The kernels widen the codes to f16 on chip (exact) and run the
+ * query through f16 for q.k (exact for |q| in [2^-14, 65504]; smaller
+ * magnitudes round to f16 subnormals); the relative term stays bf16.
+ * Current limit: shape->q_tokens must be 1 (else REL_ATTN_ERR_INVALID_ARG).
+ */
+int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q,
+                         const void* k_cache, const void* v_cache,
+                         const float* k_scale, const float* v_scale,
+                         const int32_t* block_table, const int32_t* seq_lens,
+                         const void* rel_table, int window, int num_splits,
+                         void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream);
+int rel_attn_partial_e4m3(const rel_attn_shape* shape, const void* q,
+                          const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens,
+                          const void* rel_table, int window, int num_splits,
+                          void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * rel_attn_decode_static -- rel_attn_decode without a workspace argument.
  * (An addition of this library; the pages describe nothing like it.)
  *

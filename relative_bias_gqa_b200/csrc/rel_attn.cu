@@ -12,6 +12,7 @@
 
 #include "rel_attn.h"
 #include "rel_attn_kernels.cuh"
+#include "rel_attn_fp8.cuh"
 
 namespace relattn {
 namespace {
@@ -26,6 +27,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   bool attr_set[kMaxQTokens] = {};
+  bool attr_fp8 = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -215,6 +217,17 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows) {
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// E4M3 pool: one 128-byte row per (page, head, slot), a 64-row box per page.
+bool make_map_2d_e4m3(CUtensorMap* m, const void* base, uint64_t rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim};
+  cuuint32_t box[2] = {(cuuint32_t)kHeadDim, (cuuint32_t)kPage};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_rel(CUtensorMap* m, const void* base, int NB, int Hkv, int box_rows) {
   cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)NB, (cuuint64_t)Hkv};
   cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)NB * kHeadDim * 2};
@@ -232,9 +245,11 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
       if (e.kind == kind && e.base == base && e.a == a && e.b == b) { *out = e.map; return true; }
   }
   CUtensorMap m;
-  // kinds: 0 = K pool, 1 = V pool, 2 / 3 = relative table with 136- / 128-row boxes
-  const bool ok = (kind >= 2) ? make_map_rel(&m, base, (int)a, (int)b, kind == 2 ? 136 : 128)
-                              : make_map_2d(&m, base, a);
+  // kinds: 0 = K pool, 1 = V pool, 2 / 3 = relative table with 136- / 128-row
+  // boxes, 4 / 5 = E4M3 K / V pool
+  const bool ok = (kind >= 4) ? make_map_2d_e4m3(&m, base, a)
+                  : (kind >= 2) ? make_map_rel(&m, base, (int)a, (int)b, kind == 2 ? 136 : 128)
+                                : make_map_2d(&m, base, a);
   if (!ok) return false;
   std::lock_guard<std::mutex> lk(g_cache_mu);
   MapEntry& e = g_map_cache[g_map_next++ % kMapCache];
@@ -356,10 +371,16 @@ namespace {
 int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, const void* v_cache,
             const int32_t* block_table, const int32_t* seq_lens, const void* rel_table, int window,
             int num_splits, void* out, float* lse, void* workspace, size_t workspace_bytes,
-            DecodeParams* prm, int* S_out, DeviceInfo** di_out) {
+            DecodeParams* prm, int* S_out, DeviceInfo** di_out, const float* k_scale = nullptr,
+            const float* v_scale = nullptr, bool kv_e4m3 = false) {
   // ---- validation (no CUDA call before this block passes)
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
+  if (kv_e4m3) {
+    if (shape->q_tokens != 1 || !k_scale || !v_scale ||
+        (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))
+      return REL_ATTN_ERR_INVALID_ARG;
+  }
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !rel_table || !out || !workspace)
     return REL_ATTN_ERR_INVALID_ARG;
   auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
@@ -382,8 +403,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const size_t rows = (size_t)B * T * Hq;
   memset(prm, 0, sizeof(*prm));
   const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
-  if (!cached_map(&prm->tmap_k, 0, k_cache, kv_rows, 0) ||
-      !cached_map(&prm->tmap_v, 1, v_cache, kv_rows, 0) ||
+  if (!cached_map(&prm->tmap_k, kv_e4m3 ? 4 : 0, k_cache, kv_rows, 0) ||
+      !cached_map(&prm->tmap_v, kv_e4m3 ? 5 : 1, v_cache, kv_rows, 0) ||
       !cached_map(&prm->tmap_r, group_width(6, T) == 16 ? 3 : 2, rel_table,
                   (uint64_t)shape->num_buckets, (uint64_t)Hkv))
     return REL_ATTN_ERR_CUDA;
@@ -405,6 +426,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->out_fp32 = shape->out_fp32;
   bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges, &prm->log2_ex, &prm->log_scale);
   prm->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
+  prm->k_scale = k_scale;
+  prm->v_scale = v_scale;
   *S_out = S;
   *di_out = &di;
   return REL_ATTN_OK;
@@ -424,6 +447,19 @@ int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int
     case 8: return launch_partial<8>(prm, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
+}
+
+int launch_partial_e4m3(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
+  using FC = Fp8Config;
+  auto kern = rel_attn_partial_fp8_kernel<6>;
+  if (!di.attr_fp8) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kAllocBytes) != cudaSuccess)
+      return REL_ATTN_ERR_CUDA;
+    di.attr_fp8 = true;
+  }
+  dim3 grid(S, Hkv, B);
+  kern<<<grid, FC::kThreads, FC::kAllocBytes, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
 }
 
 // LSE-merge launch; programmatic dependent launch lets it start while the
@@ -483,6 +519,39 @@ int rel_attn_partial(const rel_attn_shape* shape, const void* q, const void* k_c
                    out, lse, workspace, workspace_bytes, &prm, &S, &di);
   if (rc != REL_ATTN_OK) return rc;
   return launch_partial_any(prm, shape, S, reinterpret_cast<cudaStream_t>(stream), *di);
+}
+
+int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q, const void* k_cache,
+                         const void* v_cache, const float* k_scale, const float* v_scale,
+                         const int32_t* block_table, const int32_t* seq_lens,
+                         const void* rel_table, int window, int num_splits, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeParams prm;
+  int S = 0;
+  DeviceInfo* di = nullptr;
+  int rc = prepare(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, num_splits,
+                   out, lse, workspace, workspace_bytes, &prm, &S, &di, k_scale, v_scale, true);
+  if (rc != REL_ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = launch_partial_e4m3(prm, S, shape->batch, shape->num_kv_heads, st, *di);
+  if (rc != REL_ATTN_OK || S == 1) return rc;
+  return launch_combine(shape, S, out, lse, workspace, st);
+}
+
+int rel_attn_partial_e4m3(const rel_attn_shape* shape, const void* q, const void* k_cache,
+                          const void* v_cache, const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens,
+                          const void* rel_table, int window, int num_splits, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (num_splits < 1) return REL_ATTN_ERR_INVALID_ARG;
+  DecodeParams prm;
+  int S = 0;
+  DeviceInfo* di = nullptr;
+  int rc = prepare(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, num_splits,
+                   out, lse, workspace, workspace_bytes, &prm, &S, &di, k_scale, v_scale, true);
+  if (rc != REL_ATTN_OK) return rc;
+  return launch_partial_e4m3(prm, S, shape->batch, shape->num_kv_heads,
+                             reinterpret_cast<cudaStream_t>(stream), *di);
 }
 
 int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, float* lse,

@@ -33,6 +33,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
@@ -90,6 +91,8 @@ struct alignas(64) DecodeParams {
   int nl;               // tail buckets: bucket = ex + max{k < nl : edges[k] <= d}
   float scale_log2;     // log2(e) / sqrt(D)
   float log2_ex, log_scale;  // tail-bucket guess: (log2(d) - log2_ex) * log_scale
+  const float* k_scale;  // E4M3 KV cache only: per-KV-head scales
+  const float* v_scale;
   int edges[kMaxTailBuckets + 1];
 };
 

@@ -27,7 +27,7 @@ EXPORTED = (
     "rel_attn_decode", "rel_attn_partial", "rel_attn_combine", "rel_attn_workspace_bytes", "rel_attn_workspace_init",
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
-    "rel_attn_split_pages",
+    "rel_attn_split_pages", "rel_attn_decode_e4m3", "rel_attn_partial_e4m3",
 )
 
 
@@ -57,6 +57,11 @@ def _load():
     lib.rel_attn_partial.restype = ctypes.c_int
     lib.rel_attn_combine.argtypes = [SP, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
     lib.rel_attn_combine.restype = ctypes.c_int
+    lib.rel_attn_decode_e4m3.argtypes = [SP, P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                         P, P, P, ctypes.c_size_t, P]
+    lib.rel_attn_decode_e4m3.restype = ctypes.c_int
+    lib.rel_attn_partial_e4m3.argtypes = lib.rel_attn_decode_e4m3.argtypes
+    lib.rel_attn_partial_e4m3.restype = ctypes.c_int
     lib.rel_attn_decode_static.argtypes = [SP, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                            P, P, P]
     lib.rel_attn_decode_static.restype = ctypes.c_int
@@ -203,6 +208,43 @@ def rel_attn_decode(q, k_cache, v_cache, block_table, seq_lens, rel_table,
     return out, lse
 
 
+def rel_attn_decode_e4m3(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, rel_table,
+                         window: int = 0, num_splits: int = 0, out=None, lse=None,
+                         workspace: Optional[Workspace] = None, *, max_seq_len: int = 0,
+                         out_fp32: bool = False, exact_buckets: int = 1024,
+                         max_distance: int = 1 << 20, stream=None, with_lse: bool = True):
+    """rel_attn_decode over an E4M3 KV cache: k_codes / v_codes uint8 (or
+    float8_e4m3fn) [num_pages, Hkv, P, D], k_scale / v_scale fp32 [Hkv]."""
+    if k_codes.dtype == torch.float8_e4m3fn:
+        k_codes = k_codes.view(torch.uint8)
+    if v_codes.dtype == torch.float8_e4m3fn:
+        v_codes = v_codes.view(torch.uint8)
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_codes", k_codes, torch.uint8),
+                        ("v_codes", v_codes, torch.uint8), ("k_scale", k_scale, torch.float32),
+                        ("v_scale", v_scale, torch.float32), ("rel_table", rel_table, torch.bfloat16),
+                        ("block_table", block_table, torch.int32), ("seq_lens", seq_lens, torch.int32)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    shape = shape_of(q, k_codes, block_table, rel_table, max_seq_len=max_seq_len,
+                     out_fp32=out_fp32, exact_buckets=exact_buckets, max_distance=max_distance)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = Workspace.for_shape(shape, num_splits, q.device)
+    rc = lib.rel_attn_decode_e4m3(
+        ctypes.byref(shape), q.data_ptr(), k_codes.data_ptr(), v_codes.data_ptr(),
+        k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+        rel_table.data_ptr(), int(window), int(num_splits), out.data_ptr(),
+        lse.data_ptr() if lse is not None else None,
+        workspace.buf.data_ptr(), workspace.nbytes, _stream_ptr(stream))
+    if rc != REL_ATTN_OK:
+        raise RelAttnError(rc)
+    return out, lse
+
+
 class Prepared:
     """A decode call with every argument marshalled once (shape struct, raw
     pointers, workspace), for callers that issue the same call repeatedly.
@@ -211,7 +253,8 @@ class Prepared:
 
     def __init__(self, q, k_cache, v_cache, block_table, seq_lens, rel_table, window=0,
                  num_splits=0, *, out=None, lse=None, max_seq_len=0, out_fp32=False,
-                 exact_buckets=1024, max_distance=1 << 20, stream=None):
+                 exact_buckets=1024, max_distance=1 << 20, stream=None, k_scale=None,
+                 v_scale=None):
         self.shape = shape_of(q, k_cache, block_table, rel_table, max_seq_len=max_seq_len,
                               out_fp32=out_fp32, exact_buckets=exact_buckets,
                               max_distance=max_distance)
@@ -225,9 +268,14 @@ class Prepared:
         self.workspace = Workspace.for_shape(self.shape, num_splits, q.device)
         self.window = int(window)
         self.stream = stream
-        self._keep = (q, k_cache, v_cache, block_table, seq_lens, rel_table)
-        self._args = (q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
-                      seq_lens.data_ptr(), rel_table.data_ptr())
+        # an E4M3 KV cache (uint8 codes) comes with its per-KV-head scales
+        self.e4m3 = k_scale is not None
+        if self.e4m3 != (v_scale is not None):
+            raise ValueError("k_scale and v_scale go together")
+        self._keep = (q, k_cache, v_cache, block_table, seq_lens, rel_table, k_scale, v_scale)
+        scales = (k_scale.data_ptr(), v_scale.data_ptr()) if self.e4m3 else ()
+        self._args = (q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *scales,
+                      block_table.data_ptr(), seq_lens.data_ptr(), rel_table.data_ptr())
 
     def _common(self):
         return (ctypes.byref(self.shape), *self._args, self.window, self.num_splits,
@@ -235,13 +283,13 @@ class Prepared:
                 self.workspace.nbytes, _stream_ptr(self.stream))
 
     def decode(self):
-        rc = lib.rel_attn_decode(*self._common())
+        rc = (lib.rel_attn_decode_e4m3 if self.e4m3 else lib.rel_attn_decode)(*self._common())
         if rc != REL_ATTN_OK:
             raise RelAttnError(rc)
         return self.out, self.lse
 
     def partial(self):
-        rc = lib.rel_attn_partial(*self._common())
+        rc = (lib.rel_attn_partial_e4m3 if self.e4m3 else lib.rel_attn_partial)(*self._common())
         if rc != REL_ATTN_OK:
             raise RelAttnError(rc)
 

@@ -217,3 +217,20 @@ def poison_unused(case: DecodeCase, value: float = float("nan")) -> DecodeCase:
             k[pg, :, :head] = value
             v[pg, :, :head] = value
     return dataclasses.replace(case, k_cache=k, v_cache=v)
+
+
+def to_e4m3(case: DecodeCase):
+    """An E4M3 copy of the case's KV cache: one scale per KV head (the head's
+    largest |value| over the pool / 448, the largest finite E4M3 value) and
+    the codes of value / scale, rounded to nearest even by torch's float8
+    conversion.  Returns (k_codes uint8, v_codes uint8, k_scale fp32 [Hkv],
+    v_scale fp32 [Hkv]) on the case's device."""
+    out = []
+    for pool in (case.k_cache, case.v_cache):
+        x = pool.float()
+        amax = x.abs().amax(dim=(0, 2, 3)).clamp_min(1e-30)
+        scale = (amax / 448.0).to(torch.float32)
+        codes = (x / scale.view(1, -1, 1, 1)).to(torch.float8_e4m3fn).view(torch.uint8)
+        out.append((codes.contiguous(), scale.contiguous()))
+    (kc, ks), (vc, vs) = out
+    return kc, vc, ks, vs

@@ -1,0 +1,181 @@
+"""GPU parity of the E4M3 (FP8) KV-cache path against the fp64 oracle.
+
+The oracle dequantises the codes exactly (code value x per-KV-head scale) and
+applies the definition; the kernel widens the codes to f16 on chip.  Same
+tolerances as the bf16 path: max |out_fp32 - oracle| <= 2e-3, max |lse -
+oracle| <= 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from relative_bias_gqa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-3
+LSE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def ra():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from relative_bias_gqa_b200 import rel_attn
+    return rel_attn
+
+
+def e4m3(case):
+    kc, vc, ks, vs = W.to_e4m3(case)
+    return kc, vc, ks, vs
+
+
+def run_gpu(ra, case, codes, num_splits=0, out_fp32=True):
+    kc, vc, ks, vs = codes
+    out, lse = ra.rel_attn_decode_e4m3(case.q, kc, vc, ks, vs, case.block_table, case.seq_lens,
+                                       case.rel_table, case.window, num_splits,
+                                       max_seq_len=case.max_seq_len, out_fp32=out_fp32,
+                                       exact_buckets=case.exact_buckets,
+                                       max_distance=case.max_distance)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def run_oracle(case, codes):
+    kc, vc, ks, vs = codes
+    return oracle.rel_attn_decode_fp8kv_ref(case.q, kc, vc, ks, vs, case.block_table,
+                                            case.seq_lens, case.rel_table, case.window,
+                                            exact_buckets=case.exact_buckets,
+                                            max_distance=case.max_distance)
+
+
+def check(out, lse, ref_out, ref_lse):
+    o = out.float().cpu().numpy().astype(np.float64)
+    l = lse.cpu().numpy().astype(np.float64)
+    assert np.isfinite(o).all() and np.isfinite(l).all()
+    eo = np.abs(o - ref_out).max()
+    el = np.abs(l - ref_lse).max()
+    assert eo <= OUT_TOL and el <= LSE_TOL, (eo, el)
+
+
+def small(L, window=0, NB=1280, seed=0, Hkv=2, lens=None, **kw):
+    lens = lens if lens is not None else [L]
+    return W.make_case(seq_lens=lens, q_tokens=1, num_q_heads=6 * Hkv, num_kv_heads=Hkv,
+                       window=window, num_buckets=NB, seed=seed, extra_pages=2, **kw).to("cuda")
+
+
+SMALL = [
+    dict(L=1), dict(L=63), dict(L=64), dict(L=65), dict(L=127), dict(L=128), dict(L=129),
+    dict(L=300), dict(L=1000), dict(L=3001), dict(L=5000, seed=3),
+    dict(L=1500, window=1), dict(L=1500, window=64), dict(L=2500, window=1024),
+    dict(L=900, NB=8), dict(L=2000, NB=1030), dict(L=200, window=1024, NB=1024),
+    dict(L=6000, NB=364, exact_buckets=64, max_distance=5000),
+]
+
+
+@pytest.mark.parametrize("kw", SMALL, ids=[str(k) for k in SMALL])
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_small_cases(ra, kw, splits):
+    case = small(**kw)
+    codes = e4m3(case)
+    check(*run_gpu(ra, case, codes, splits), *run_oracle(case, codes))
+
+
+def test_batched_mixed_lengths(ra):
+    case = small(0, Hkv=3, lens=[5, 64, 65, 300, 1111, 2049, 129, 2])
+    codes = e4m3(case)
+    ref = run_oracle(case, codes)
+    for splits in (1, 2, 5, 0):
+        check(*run_gpu(ra, case, codes, splits), *ref)
+
+
+def test_split_count_invariance(ra):
+    case = small(20000)
+    codes = e4m3(case)
+    ref = run_oracle(case, codes)
+    for s in (1, 2, 3, 5, 8, 13, 18, 37, 64, 157):
+        check(*run_gpu(ra, case, codes, s), *ref)
+
+
+def test_bf16_output_is_rounded_fp32(ra):
+    case = small(2600)
+    codes = e4m3(case)
+    for splits in (1, 4):
+        o32, l32 = run_gpu(ra, case, codes, splits, out_fp32=True)
+        o16, l16 = run_gpu(ra, case, codes, splits, out_fp32=False)
+        assert torch.equal(o32.to(torch.bfloat16), o16)
+        assert torch.equal(l32, l16)
+
+
+def test_nan_codes_in_unseen_slots_do_not_matter(ra):
+    """E4M3 NaN codes (0x7F) in every cache slot no query can see."""
+    for kw in (dict(L=3001), dict(L=2500, window=1024, NB=1024), dict(L=1500, window=100)):
+        case = small(**kw)
+        kc, vc, ks, vs = e4m3(case)
+        ref = run_oracle(case, (kc, vc, ks, vs))
+        L = int(case.seq_lens[0])
+        lo = max(0, L - 1 - case.window + 1) if case.window > 0 else 0
+        seen = torch.zeros(kc.shape[0], kc.shape[2], dtype=torch.bool)
+        bt = case.block_table[0].cpu()
+        for j in range(lo, L):
+            seen[int(bt[j // 64]), j % 64] = True
+        mask = (~seen).to(kc.device)[:, None, :, None].expand_as(kc)
+        kp, vp = kc.clone(), vc.clone()
+        kp[mask] = 0x7F
+        vp[mask] = 0x7F
+        for splits in (1, 4):
+            clean = run_gpu(ra, case, (kc, vc, ks, vs), splits)
+            bad = run_gpu(ra, case, (kp, vp, ks, vs), splits)
+            assert torch.equal(clean[0], bad[0]) and torch.equal(clean[1], bad[1])
+            check(*bad, *ref)
+
+
+def test_scales_are_per_kv_head(ra):
+    """Distinct scales per head: doubling head 1's V scale doubles only its rows."""
+    case = small(3000)
+    kc, vc, ks, vs = e4m3(case)
+    o1, l1 = run_gpu(ra, case, (kc, vc, ks, vs), 3)
+    vs2 = vs.clone()
+    vs2[1] *= 2
+    o2, l2 = run_gpu(ra, case, (kc, vc, ks, vs2), 3)
+    assert torch.equal(o1[:, :, :6], o2[:, :, :6])
+    assert torch.allclose(o2[:, :, 6:], 2 * o1[:, :, 6:], rtol=1e-6, atol=0)
+    assert torch.equal(l1, l2)
+
+
+def test_full_100k(ra):
+    case = W.make_workload("full_100k", seed=0, device="cuda")
+    codes = e4m3(case)
+    ref = run_oracle(case, codes)
+    for s in (1, 7, 18, 37, 148, 0):
+        check(*run_gpu(ra, case, codes, s), *ref)
+
+
+def test_sliding_100k(ra):
+    case = W.make_workload("sliding_100k", seed=1, device="cuda")
+    codes = e4m3(case)
+    ref = run_oracle(case, codes)
+    for s in (1, 4, 0):
+        check(*run_gpu(ra, case, codes, s), *ref)
+
+
+def test_rejects_several_query_tokens_and_missing_scales(ra):
+    case = W.make_case(seq_lens=[300], q_tokens=2, num_q_heads=12, num_kv_heads=2,
+                       seed=0).to("cuda")
+    kc, vc, ks, vs = e4m3(case)
+    with pytest.raises(ra.RelAttnError) as e:
+        run_gpu(ra, case, (kc, vc, ks, vs), 1)
+    assert e.value.code == ra.REL_ATTN_ERR_INVALID_ARG
+    import ctypes
+    one = small(300)
+    kc, vc, ks, vs = e4m3(one)
+    shape = ra.shape_of(one.q, kc, one.block_table, one.rel_table, max_seq_len=300)
+    ws = ra.Workspace.for_shape(shape, 1, one.q.device)
+    out = torch.empty_like(one.q)
+    rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(shape), one.q.data_ptr(), kc.data_ptr(),
+                                     vc.data_ptr(), None, vs.data_ptr(), one.block_table.data_ptr(),
+                                     one.seq_lens.data_ptr(), one.rel_table.data_ptr(), 0, 1,
+                                     out.data_ptr(), None, ws.buf.data_ptr(), ws.nbytes, None)
+    assert rc == ra.REL_ATTN_ERR_INVALID_ARG
