@@ -16,8 +16,8 @@
 //   warps 2..9    two softmax groups alternating tiles (as the one-token bf16
 //                 kernel), P in f16 hi + lo parts.
 //   warps 10..13  converter: one thread per key row widens the staged E4M3 K
-//                 and V rows to f16 (cvt.rn.f16x2.e4m3x2) into the MMA's
-//                 128B-swizzled layouts, zeroing V rows no query may see.
+//                 and V rows to f16 (cvt.rn.f16x2.e4m3x2, exact) into the
+//                 MMA's 128B-swizzled layouts, zeroing V rows no query may see.
 // The K scale multiplies the S logits, the V scale the final output.  The
 // softmax's lazy reference max lets P grow to 2^14 here (f16 range).
 #pragma once
@@ -63,10 +63,10 @@ struct Fp8Config {
   static_assert(oXR >= NG * RG * 128 * 4 * 2 + NG * RG * 4 * 2, "epilogue exchange area");
 };
 
-// E4M3 pair -> f16x2 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+// E4M3 pair (low 16 bits) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
   uint32_t r;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)v));
   return r;
 }
 
@@ -88,6 +88,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
@@ -252,6 +253,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         ptx::mbar_arrive_expect_tx(v8full(ti % V8S), tp.npg * FC::k8PageBytes);
         ptx::tma_load_2d(st, &p.tmap_v, v8full(ti % V8S), 0, row0, pol);
         if (tp.npg > 1) ptx::tma_load_2d(st + FC::k8PageBytes, &p.tmap_v, v8full(ti % V8S), 0, row1, pol);
+        RELATTN_TRACE(0, ti);
       }
       ++nv;
     }
@@ -269,56 +271,62 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     }
   }
   // ------------------------------------------------------------ converter
+  // Order K(0), then per tile K(i+1) before V(i): K(i+1) needs only S(i) to
+  // have read the K16 slot, V(i) needs P.V(i-1) to have read the V16 slot,
+  // so the K side runs a tile ahead and S(i+1) and its softmax never wait
+  // behind the P.V chain.
   else if (warp >= 10) {
     const int kc = tid - 320;                     // key row of the tile
     const int sw = kc & 7;
-    bool ok = true;
-    for (int ti = 0; ti < g.ntiles && ok; ++ti) {
-      const int npg = min(2, g.sp_end - (g.sp_begin + 2 * ti));
-      const bool loaded = kc < npg * kPage;
-      const int j = (g.sp_begin + 2 * ti) * kPage + kc;
-      const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
-      // one E4M3 row (128 B, 8 swizzled 16-byte chunks) -> f16 row (two 128 B
-      // halves of the K-major / MN-major 128B-swizzled tile)
-      auto widen = [&](uint32_t src_slot, uint8_t* dst_tile, bool zero) {
-        const uint8_t* src = smem + (src_slot - sbase) + kc * 128;
+    // one E4M3 row (128 B, 8 swizzled 16-byte chunks) -> f16 row (two 128 B
+    // halves of the K-major / MN-major 128B-swizzled tile)
+    auto widen = [&](uint32_t src_slot, uint8_t* dst_tile, bool zero) {
+      const uint8_t* src = smem + (src_slot - sbase) + kc * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 w = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-          if (!zero) {
-            w = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
-            const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-            uint32_t o[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              o[2 * q] = e4m3x2_to_f16x2((uint16_t)(in[q] & 0xffffu));
-              o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(in[q] >> 16));
-            }
-            lo4 = make_uint4(o[0], o[1], o[2], o[3]);
-            hi4 = make_uint4(o[4], o[5], o[6], o[7]);
-          }
-          // 16 dims 16c..16c+15 -> half c/4, 16-byte chunks 2(c%4), 2(c%4)+1
-          uint8_t* row = dst_tile + (c >> 2) * kHalfTileBytes + kc * 128;
-          *reinterpret_cast<uint4*>(row + (((2 * (c & 3)) ^ sw) << 4)) = lo4;
-          *reinterpret_cast<uint4*>(row + (((2 * (c & 3) + 1) ^ sw) << 4)) = hi4;
+      for (int c = 0; c < 8; ++c) {
+        uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
+        if (!zero) {
+          const uint4 w = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+          lo4 = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
+                           e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
+          hi4 = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
+                           e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
         }
-      };
-      // K
-      ok = ptx::mbar_wait(k8full(ti % K8S), (ti / K8S) & 1, abort_flag, tlim) &&
-           ptx::mbar_wait(kf_empty, (ti & 1) ^ 1, abort_flag, tlim);
-      if (!ok) break;
-      if (loaded) widen(sbase + FC::oK8 + (ti % K8S) * FC::k8TileBytes, smem + FC::oKF, false);
+        // 16 dims 16c..16c+15 -> half c/4, 16-byte chunks 2(c%4), 2(c%4)+1
+        uint8_t* row = dst_tile + (c >> 2) * kHalfTileBytes + kc * 128;
+        *reinterpret_cast<uint4*>(row + (((2 * (c & 3)) ^ sw) << 4)) = lo4;
+        *reinterpret_cast<uint4*>(row + (((2 * (c & 3) + 1) ^ sw) << 4)) = hi4;
+      }
+    };
+    auto tile_pages = [&](int ti) { return min(2, g.sp_end - (g.sp_begin + 2 * ti)); };
+    auto convert_k = [&](int ti) -> bool {
+      if (!ptx::mbar_wait(k8full(ti % K8S), (ti / K8S) & 1, abort_flag, tlim) ||
+          !ptx::mbar_wait(kf_empty, (ti & 1) ^ 1, abort_flag, tlim))
+        return false;
+      if (kc < tile_pages(ti) * kPage) widen(sbase + FC::oK8 + (ti % K8S) * FC::k8TileBytes, smem + FC::oKF, false);
       ptx::fence_proxy_async_smem();
+      if (kc == 0) RELATTN_TRACE(2, ti);
       ptx::mbar_arrive(kf_full);
       ptx::mbar_arrive(k8empty(ti % K8S));
-      // V (rows no query may see are zeroed: 0 * NaN must not reach P.V)
-      ok = ptx::mbar_wait(v8full(ti % V8S), (ti / V8S) & 1, abort_flag, tlim) &&
-           ptx::mbar_wait(vf_empty, (ti & 1) ^ 1, abort_flag, tlim);
-      if (!ok) break;
+      return true;
+    };
+    auto convert_v = [&](int ti) -> bool {
+      // rows no query may see are zeroed: 0 * NaN must not reach P.V
+      const int j = (g.sp_begin + 2 * ti) * kPage + kc;
+      const bool any_valid = kc < tile_pages(ti) * kPage && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
+      if (!ptx::mbar_wait(v8full(ti % V8S), (ti / V8S) & 1, abort_flag, tlim) ||
+          !ptx::mbar_wait(vf_empty, (ti & 1) ^ 1, abort_flag, tlim))
+        return false;
       widen(sbase + FC::oV8 + (ti % V8S) * FC::k8TileBytes, smem + FC::oVF, !any_valid);
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(vf_full);
       ptx::mbar_arrive(v8empty(ti % V8S));
+      return true;
+    };
+    bool ok = convert_k(0);
+    for (int ti = 0; ti < g.ntiles && ok; ++ti) {
+      if (ti + 1 < g.ntiles) ok = convert_k(ti + 1);
+      ok = ok && convert_v(ti);
     }
   }
   // ------------------------------------------------------------ MMA issuer
@@ -342,6 +350,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
         if (!ptx::mbar_wait(vf_full, j & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
+        RELATTN_TRACE(3, j);
         const uint64_t pbd = pdesc + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -354,13 +363,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       for (int ti = 0; ti < g.ntiles; ++ti) {
         const int gq = ti & 1;
         const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
-        // P.V of the previous tile frees the V16 slot: issue it first unless
-        // this tile's K16 is already there (then S first, so softmax starts).
-        bool pv_pending = i > 0;
-        if (pv_pending && !ptx::mbar_try_wait(kf_full, i & 1)) {
-          if (!(ok = issue_pv(i - 1))) break;
-          pv_pending = false;
-        }
+        // S(i) first, then P.V(i-1): the converter widens K(i) before
+        // V(i-1), so S(i) never waits on the P.V chain.
+        const bool pv_pending = i > 0;
         if (tp.chunk) {
           ok = ptx::mbar_wait(xr_full, nx & 1, abort_flag, tlim) &&
                ptx::mbar_wait(x_empty + 8u * gq, (cg[gq] & 1) ^ 1, abort_flag, tlim);
@@ -381,6 +386,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
              ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
         if (!ok) break;
         ptx::tc_fence_after();
+        RELATTN_TRACE(1, i);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t ko = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
@@ -468,6 +474,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       const bool okw = ptx::mbar_wait(s_full + 8u * (i & 1), (i >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
+        RELATTN_TRACE(4, i);
         ptx::tmem_ld8(tS + lane_off + (i & 1) * N, s);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
@@ -517,6 +524,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int r = 0; r < RG; ++r) alpha_r[r] = 1.f;
       }
+      RELATTN_TRACE(5, i);
       // ---- P = exp2(x - m_ref) as f16 hi + lo parts, stacked [P_hi; P_lo],
       //      MN-major without swizzle (8-row x 16-byte core matrices)
       {
@@ -541,7 +549,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
+      RELATTN_TRACE(6, i);
       process_o(i);                            // this group's next tile is i + 2
+      RELATTN_TRACE(7, i);
       ++li;
     }
     ptx::pdl_launch_dependents();
@@ -600,6 +610,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   ptx::tc_fence_before();
   __syncthreads();
   if (tid == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);
+  RELATTN_TRACE(17, 0);
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);
