@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--kv-dtype", choices=("bf16", "e4m3"), default="bf16",
+                    help="KV-cache format: bf16, or E4M3 codes with per-KV-head scales")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -68,10 +70,11 @@ def kernel_source_hash() -> str:
 
 
 # ------------------------------------------------------------ bookkeeping
-def algorithmic_bytes(case, bucket_fn, out_bytes=2):
-    """Bytes the call must move: visible K/V rows once, the relative-table
-    rows [0, bucket(max distance)] of every KV head once, q, out, lse, the
-    block-table entries read and seq_lens."""
+def algorithmic_bytes(case, bucket_fn, out_bytes=2, kv_elem_bytes=2):
+    """Bytes the call must move: visible K/V rows once (kv_elem_bytes per
+    element: 2 for bf16, 1 for E4M3 plus the per-head scales), the
+    relative-table rows [0, bucket(max distance)] of every KV head once, q,
+    out, lse, the block-table entries read and seq_lens."""
     lens = case.seq_lens.cpu().tolist()
     T, Hq, Hkv, D, P = (case.q_tokens, case.num_q_heads, case.num_kv_heads,
                         case.head_dim, case.page_size)
@@ -81,12 +84,14 @@ def algorithmic_bytes(case, bucket_fn, out_bytes=2):
     d_max = 0
     for L in lens:
         lo = max(0, L - T - W + 1) if W > 0 else 0
-        kv += (L - lo) * Hkv * D * 2 * 2
+        kv += (L - lo) * Hkv * D * 2 * kv_elem_bytes
         pages += (L - 1) // P - lo // P + 1
         d_max = max(d_max, min(W - 1, L - 1) if W > 0 else L - 1)
     r_rows = bucket_fn(d_max) + 1
     rel = r_rows * Hkv * D * 2
     small = len(lens) * T * Hq * (D * 2 + D * out_bytes + 4) + pages * 4 + len(lens) * 4
+    if kv_elem_bytes == 1:
+        small += 2 * Hkv * 4                          # K and V scales
     return kv + rel + small, dict(kv=kv, rel=rel, other=small)
 
 
@@ -235,12 +240,18 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     case = workloads.make_workload(args.workload, seed=args.seed + rank, device=dev)
-    prep = rel_attn.Prepared(case.q, case.k_cache, case.v_cache, case.block_table, case.seq_lens,
-                             case.rel_table, case.window, args.num_splits,
-                             max_seq_len=case.max_seq_len, out_fp32=False)
+    e4m3 = args.kv_dtype == "e4m3"
+    if e4m3:
+        kc, vc, ks, vs = workloads.to_e4m3(case)
+        kv_args = dict(k_cache=kc, v_cache=vc, scales=dict(k_scale=ks, v_scale=vs))
+    else:
+        kv_args = dict(k_cache=case.k_cache, v_cache=case.v_cache, scales={})
+    prep = rel_attn.Prepared(case.q, kv_args["k_cache"], kv_args["v_cache"], case.block_table,
+                             case.seq_lens, case.rel_table, case.window, args.num_splits,
+                             max_seq_len=case.max_seq_len, out_fp32=False, **kv_args["scales"])
     S = prep.num_splits
     bucket = lambda d: rel_attn.rel_attn_bucket(prep.shape, d)
-    nbytes, parts = algorithmic_bytes(case, bucket)
+    nbytes, parts = algorithmic_bytes(case, bucket, kv_elem_bytes=1 if e4m3 else 2)
     props = torch.cuda.get_device_properties(dev)
     flush = torch.empty(2 * max(props.L2_cache_size, 64 << 20), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -322,9 +333,9 @@ def run_ours(args, rank, world, local_rank):
     out_parts = (prep.out, prep.lse)
     d_res, (d_out, d_lse) = packed(out_parts, "dev")
     h_res, _ = packed(out_parts, "pin")
-    prep_e2e = rel_attn.Prepared(d_q, case.k_cache, case.v_cache, d_bt, d_sl, case.rel_table,
-                                 case.window, S, out=d_out, lse=d_lse,
-                                 max_seq_len=case.max_seq_len, out_fp32=False)
+    prep_e2e = rel_attn.Prepared(d_q, kv_args["k_cache"], kv_args["v_cache"], d_bt, d_sl,
+                                 case.rel_table, case.window, S, out=d_out, lse=d_lse,
+                                 max_seq_len=case.max_seq_len, out_fp32=False, **kv_args["scales"])
     Ke = min(K, 2000)
     eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
     for i in range(Ke):
@@ -365,8 +376,11 @@ def run_ours(args, rank, world, local_rank):
             "us_partial_kernel": round(mean_part * 1e3, 2),
             "us_combine_kernel_after_event": round(statistics.fmean(t_comb) * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) relative table)",
-            "config": {"workload": args.workload, "batch": case.batch, "q_tokens": case.q_tokens,
+            "dtype": "bf16" if not e4m3 else "bf16 q, e4m3 kv (f16 on chip)",
+            "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) relative table)" +
+                    ("; K/V quantised to E4M3 with per-KV-head amax/448 scales" if e4m3 else ""),
+            "config": {"workload": args.workload, "kv_dtype": args.kv_dtype,
+                       "batch": case.batch, "q_tokens": case.q_tokens,
                        "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
                        "head_dim": case.head_dim, "seq_lens_max": case.max_seq_len,
                        "window": case.window, "num_buckets": case.num_buckets,
@@ -378,8 +392,8 @@ def run_ours(args, rank, world, local_rank):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                          else "fallback 6.65 TB/s",
-                         "kernel": "rel_attn_partial_kernel",
-                         "traffic": load_traffic(src_hash, args.workload),
+                         "kernel": "rel_attn_partial_fp8_kernel" if e4m3 else "rel_attn_partial_kernel",
+                         "traffic": load_traffic(src_hash, args.workload + ("_e4m3" if e4m3 else "")),
                          "frac_of_8TBps_nominal": round(achieved / 8000.0, 4)},
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "us_per_call": round(statistics.fmean(t_e2e) * 1e3, 2),
