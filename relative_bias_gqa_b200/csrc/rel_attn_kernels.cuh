@@ -118,9 +118,11 @@ struct KernelConfig {
   static constexpr int kRows = (N == 16) ? 128 : 136;
   static constexpr int kRHalfBytes = kRows * 128;
   static constexpr int kKSlotBytes = 2 * kRHalfBytes;          // >= one K tile (32 KB)
-  static constexpr int kKSlots = (N == 16) ? 3 : 2;
-  static constexpr int kVSlots = (N == 16) ? 3 : (N == 32 ? 3 : 2);
-  static constexpr int kVLag = (N == 16) ? 1 : 0;               // V issued this many tiles after K
+  // K slots turn over fast (freed by the S MMA), V slots slowly (held until
+  // P.V), so the one-token instance gives V four of its six 32 KB slots.
+  static constexpr int kKSlots = 2;
+  static constexpr int kVSlots = (N == 16) ? 4 : (N == 32 ? 3 : 2);
+  static constexpr int kVLag = 0;                               // V issued this many tiles after K
   // Relative-table gather stride: odd for conflict-free gathers.  The N = 16
   // instance serves at most 6 live rows.
   static constexpr int kYStride = (N == 16) ? 7 : N + 1;
