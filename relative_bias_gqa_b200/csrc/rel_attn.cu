@@ -50,12 +50,12 @@ bool encode_fn_ready() {
 }
 
 // Group width N (GQA group x query tokens, padded to the MMA N step of 16).
-// The 16-wide instance serves one token (6 rows); 32 and 48 hold two 8-aligned
-// row blocks, one per softmax group.
+// The 16-wide instance serves one token (6 rows); 32 and 48 hold one row block
+// per softmax group (blocks 8-aligned, or 4-aligned where 8 does not fit).
 int group_width(int G, int T) {
   const int nq = G * T;
   if (nq <= 6) return 16;
-  if (nq <= 24) return 32;     // two groups' rows, each block 8-aligned, in 32 slots
+  if (nq <= 24) return 32;     // two groups' rows, 8-aligned blocks, in 32 slots
   if (nq <= 48) return 48;
   return 0;
 }
@@ -261,7 +261,7 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
 template <int T>
 int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
   constexpr int N = (T == 1) ? 16 : (T <= 4 ? 32 : 48);              // group width, as group_width()
-  constexpr int NG = 2;
+  constexpr int NG = softmax_groups(T);
   constexpr int slot = T - 1;
   using KC = KernelConfig<N, NG>;
   auto kern = rel_attn_partial_kernel<N, 6, NG, T>;

@@ -11,12 +11,14 @@
 //                 S^T = K . Q^T           (128 keys x N)
 //                 X^T = R_chunk . Q^T     (136 relative rows x N)
 //                 O^T = V^T . P^T         (128 dims x N)
-//   softmax     NG groups of 4 warps (one key / one head-dim lane per thread);
-//               with two groups, group g takes the tiles i with i % 2 == g, so
-//               two tiles' softmax run at once (each group keeps its own
-//               running max / sum / output and its own relative-row chunk;
-//               the two partial states are merged by LSE at the end).  Per
-//               tile: tcgen05.ld of S^T, relative term sheared into place
+//   softmax     NG groups of 4 warps (one key / one head-dim lane per thread).
+//               One token: two groups, group g takes the tiles i with
+//               i % 2 == g, so two tiles' softmax run at once (each group
+//               keeps its own running max / sum / output and its own
+//               relative-row chunk; the two partial states are merged by LSE
+//               at the end).  Several tokens: every group takes every tile
+//               and its own block of the query rows (two groups up to five
+//               tokens, four beyond).  Per tile: tcgen05.ld of S^T, relative term sheared into place
 //               through a shared-memory table indexed by bucket(distance),
 //               masks, fp32 online softmax in the log2 domain, P to shared
 //               memory (bf16 hi + lo, 128B-swizzled), O^T tile accumulated in
@@ -59,6 +61,14 @@ constexpr int kPage = 64;
 constexpr int kTileKeys = 128;                 // two pages per tile
 constexpr int kMaxTailBuckets = 512;           // log buckets supported
 constexpr int kSoftmaxThreads = 128;           // one softmax group
+// named barriers: 1 .. NG one per softmax group, then these two
+constexpr int kBarSoftmaxAll = 5;              // every softmax thread (epilogue)
+constexpr int kBarSetup = 6;                   // every warp but the producer (prologue)
+// Softmax groups of the instance for T query tokens: two for up to five
+// tokens, four beyond (each group then carries at most 12 rows of S^T, so a
+// thread's per-tile work halves and every SM sub-partition runs four softmax
+// warps to hide each other's latencies).
+__host__ __device__ constexpr int softmax_groups(int T) { return T >= 6 ? 4 : 2; }
 constexpr int kVSlotBytes = 32768;             // V tile: 128 keys x 128 dims bf16
 constexpr int kHalfTileBytes = 16384;          // 128 rows x 128 B (one 64-dim half)
 constexpr int kPageHalfBytes = 8192;           // 64 rows x 128 B
@@ -106,13 +116,13 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 template <int N, int NG>
 struct KernelConfig {
   // N = 16 (one token): the softmax groups alternate tiles, each with all the
-  // rows.  N = 32 / 48 (2..8 tokens): both groups take every tile, each with
+  // rows.  N = 32 / 48 (2..8 tokens): every group takes every tile, each with
   // its own block of rows (a column split of S^T, X^T and O^T).
   static constexpr bool kAlt = (N == 16);
   static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
   static constexpr int kConsumers = kAlt ? kSoftmaxThreads : kSoftmaxThreads * NG;  // arrivals per tile
   static constexpr int kXTables = kAlt ? NG : 1;               // relative chunks in flight (X, Y)
-  static constexpr int kGR = kAlt ? N : N / 2;                 // row capacity of a group
+  static constexpr int kGR = kAlt ? N : N / NG;                // row capacity of a group
   // relative rows per chunk: 128 cover one 128-key tile for one token; with
   // T tokens a tile needs 127 + T rows
   static constexpr int kRows = (N == 16) ? 128 : 136;
@@ -154,6 +164,25 @@ struct KernelConfig {
   static_assert(kKSlotBytes >= 2 * kHalfTileBytes && oV % 1024 == 0 && oQ % 1024 == 0,
                 "slot layout");
   static_assert(oV >= NG * kGR * 128 * 4 * 2 + NG * kGR * 4 * 2, "epilogue exchange area");
+};
+
+// Column split of the query rows among NG softmax groups (T >= 2): group q
+// takes tokens [tok_begin(q), tok_begin(q+1)) and the query slots from
+// slot(q, A) on, slots packed with alignment A = 8 where that fits in N, else
+// 4 (a 4-aligned group reads its tensor-memory columns from the 8-aligned
+// column below and shifts by four).
+template <int T, int G, int NG>
+struct ColSplit {
+  __host__ __device__ static constexpr int tok_begin(int q) { return q * T / NG; }
+  __host__ __device__ static constexpr int rows(int q) { return (tok_begin(q + 1) - tok_begin(q)) * G; }
+  __host__ __device__ static constexpr int slot(int q, int a) {
+    int s = 0;
+    for (int u = 0; u < q; ++u) s = align_up(s + rows(u), a);
+    return s;
+  }
+  __host__ __device__ static constexpr int end(int a) { return align_up(slot(NG - 1, a) + rows(NG - 1), a); }
+  __host__ __device__ static constexpr int align(int n) { return end(8) <= n ? 8 : 4; }
+  static constexpr int kMaxRows = (T + NG - 1) / NG * G;
 };
 
 // Per-CTA geometry shared by the three roles.
@@ -342,18 +371,17 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const int warp = tid >> 5, lane = tid & 31;
   const int s_idx = RELATTN_SPLIT_OF_BLOCK(blockIdx.x), h = RELATTN_HEAD_OF_BLOCK(blockIdx.y), b = blockIdx.z;
   constexpr int NQ = T * G;
-  // rows per softmax group: all NQ when the groups alternate tiles; else
-  // group 0 takes the first TA tokens and group 1 the other TB, group 1's
-  // rows starting at query slot kSlot1 (8-aligned, so no 8-row block of P is
-  // shared by the groups)
-  constexpr int TA = KC::kAlt ? T : (T + 1) / 2;
-  constexpr int TB = KC::kAlt ? T : T - TA;
-  constexpr int RG = TA * G;
+  // rows per softmax group: all NQ when the groups alternate tiles, else the
+  // group's block of the column split (at most RG rows, TG tokens)
+  using CSp = ColSplit<T, G, NG>;
+  constexpr int kAlign = KC::kAlt ? 8 : CSp::align(N);
+  constexpr int RG = KC::kAlt ? NQ : CSp::kMaxRows;
+  constexpr int TG = RG / G;
   constexpr int RG8 = (RG + 7) / 8;
-  constexpr int kSlot1 = KC::kAlt ? 0 : align_up(RG, 8);
-  constexpr bool kEvenSplit = KC::kAlt || TA == TB;
-  static_assert(NG == 2, "two softmax groups");
-  static_assert(KC::kAlt ? NQ <= N : (kSlot1 + TB * G <= N && RG <= KC::kGR), "group width");
+  constexpr int RGL8 = (kAlign == 8) ? RG8 : (RG + 4 + 7) / 8;   // 8-column loads per row block
+  constexpr bool kEvenSplit = KC::kAlt || T % NG == 0;
+  static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(T) && CSp::end(kAlign) <= N &&
+                                                   RG <= KC::kGR), "group width");
   RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
@@ -440,14 +468,22 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       const int st = tid - 64;
       const int nst = kSoftmaxThreads * NG;
       // Q group tile, 128B-swizzled K-major: query slot n holds (token t,
-      // head gg) with n = t*G + gg, except that with column-split groups
-      // group 1's tokens start at slot kSlot1; other slots are zero.
+      // head gg) with n = t*G + gg, except that column-split groups start
+      // their tokens at their own slots; other slots are zero.
       for (int u = st; u < N * 16; u += nst) {
         const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
         uint4 v = make_uint4(0, 0, 0, 0);
-        const int nl = (n >= kSlot1 && !KC::kAlt) ? n - kSlot1 + TA * G : n;   // row t*G + gg
-        const bool used = KC::kAlt ? n < NQ : (n < kSlot1 ? n < RG : nl < NQ);
-        if (used) {
+        int nl = -1;                                      // row t*G + gg of slot n
+        if constexpr (KC::kAlt) {
+          nl = n < NQ ? n : -1;
+        } else {
+#pragma unroll
+          for (int q = 0; q < NG; ++q) {
+            const int s0 = CSp::slot(q, kAlign);
+            if (n >= s0 && n < s0 + CSp::rows(q)) nl = CSp::tok_begin(q) * G + n - s0;
+          }
+        }
+        if (nl >= 0) {
           const int t = nl / G, gg = nl % G;
           const __nv_bfloat16* src = p.q + ((size_t)(b * T + t) * p.Hq + h * G + gg) * kHeadDim
                                      + half * 64 + w16 * 8;
@@ -460,7 +496,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       ptx::fence_proxy_async_smem();
     }
     ptx::tc_fence_before();
-    ptx::bar_sync_or(4, KC::kThreads - 32, false);   // every warp but the producer
+    ptx::bar_sync_or(kBarSetup, KC::kThreads - 32, false);   // every warp but the producer
     ptx::tc_fence_after();
     tmem = *tmem_holder;
   }
@@ -525,6 +561,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
             ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
           }
+          RELATTN_TRACE(2, ti);
         }
         ++k;
       }
@@ -662,15 +699,45 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     const int bar_id = 1 + grp;
     const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
     // this group's rows: query slots [slot0, slot0 + RG), tokens from tok0;
-    // `nrows` of them are live (fewer than RG only for group 1 at odd T)
-    const int slot0 = KC::kAlt ? 0 : grp * kSlot1;
-    const int tok0 = KC::kAlt ? 0 : grp * TA;
-    const int nrows = KC::kAlt ? NQ : (grp ? TB * G : TA * G);
+    // `nrows` of them are live (fewer than RG only when T % NG != 0)
+    int slot0 = 0, tok0 = 0, nrows = NQ;
+    if constexpr (!KC::kAlt) {
+      slot0 = CSp::slot(0, kAlign);
+      tok0 = CSp::tok_begin(0);
+      nrows = CSp::rows(0);
+#pragma unroll
+      for (int q = 1; q < NG; ++q) {
+        if (grp == q) {
+          slot0 = CSp::slot(q, kAlign);
+          tok0 = CSp::tok_begin(q);
+          nrows = CSp::rows(q);
+        }
+      }
+    }
     auto live = [&](int r) { return r < RG && (kEvenSplit || r < nrows); };
     float* Y = reinterpret_cast<float*>(smem + KC::oY + (KC::kAlt ? grp : 0) * KC::kYBytes);
     float* red = reinterpret_cast<float*>(smem + KC::oRed) + grp * 2 * 4 * KC::kGR;
     float* alpha_buf = reinterpret_cast<float*>(smem + KC::oAlpha) + grp * 2 * KC::kGR;
-    const uint32_t tXg = tX(KC::kAlt ? grp : 0) + lane_off + slot0;
+    const uint32_t tXg = tX(KC::kAlt ? grp : 0) + lane_off;
+    // This group's RG columns of a tensor-memory block whose query slot 0 is
+    // at column `ta`, for this thread's lane.  A 4-aligned block is read from
+    // the 8-aligned column below it and shifted down by four.
+    const int cbase = slot0 & ~7;
+    const bool sh4 = (kAlign == 4) && (slot0 & 4);
+    auto ld_rows = [&](uint32_t ta, float (&v)[RG8 * 8]) {
+      if constexpr (kAlign == 8) {
+#pragma unroll
+        for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(ta + slot0 + q8 * 8, v + q8 * 8);
+        ptx::tmem_wait_ld();
+      } else {
+        float raw[RGL8 * 8];
+#pragma unroll
+        for (int q8 = 0; q8 < RGL8; ++q8) ptx::tmem_ld8(ta + cbase + q8 * 8, raw + q8 * 8);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int r = 0; r < RG8 * 8; ++r) v[r] = (r + 4 < RGL8 * 8 && sh4) ? raw[r + 4] : raw[r];
+      }
+    };
     // per-row running state: l (this thread's keys), O (this thread's head-dim
     // lane), reference max; alpha_r carries this tile's rescale factors when
     // O is taken right away (alternating groups)
@@ -691,12 +758,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       const bool okw = ptx::mbar_wait(o_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N + slot0;
+        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {          // O^T from P_hi, then from P_lo
-#pragma unroll
-          for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(ob + part * N + q8 * 8, ov + q8 * 8);
-          ptx::tmem_wait_ld();
+          ld_rows(ob + part * N, ov);
 #pragma unroll
           for (int r = 0; r < RG; ++r)
             if (live(r)) o_acc[r] = part ? o_acc[r] + ov[r] : fmaf(o_acc[r], al[r], ov[r]);
@@ -723,16 +788,12 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           if (okw) {
             float xv[RG8 * 8];
             ptx::tc_fence_after();
-#pragma unroll
-            for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(tXg + q8 * 8, xv + q8 * 8);
-            ptx::tmem_wait_ld();
+            ld_rows(tXg, xv);
 #pragma unroll
             for (int r = 0; r < RG; ++r)
               if (live(r)) Y[kl * YS + slot0 + r] = xv[r];
             if (ROWS > 128 && sp == 3) {         // rows 128..135 come from lanes 120..127 of X1
-#pragma unroll
-              for (int q8 = 0; q8 < RG8; ++q8) ptx::tmem_ld8(tXg + N + q8 * 8, xv + q8 * 8);
-              ptx::tmem_wait_ld();
+              ld_rows(tXg + N, xv);
               if (lane >= 24) {
 #pragma unroll
                 for (int r = 0; r < RG; ++r)
@@ -756,10 +817,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if (okw) {
         ptx::tc_fence_after();
         RELATTN_TRACE(4, i);
-#pragma unroll
-        for (int q8 = 0; q8 < RG8; ++q8)
-          ptx::tmem_ld8(tS + lane_off + (i & 1) * N + slot0 + q8 * 8, s + q8 * 8);
-        ptx::tmem_wait_ld();
+        ld_rows(tS + lane_off + (i & 1) * N, s);
         ptx::tc_fence_before();
       }
       ptx::mbar_arrive(s_empty + 8u * (i & 1));
@@ -774,7 +832,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) e_hi[m] = s_edges[max(tp.k_hi - m, 0)];
 #pragma unroll
-      for (int tt = 0; tt < TA; ++tt) {
+      for (int tt = 0; tt < TG; ++tt) {
         if (!kEvenSplit && tt * G >= nrows) break;
         const int d = d0 + tok0 + tt;
         const bool v = loaded && d >= 0 && (g.W <= 0 || d < g.W);
@@ -838,20 +896,24 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       // ---- P = exp2(x - m_ref) as bf16 hi + lo parts (~16 significant bits in
       //      the P.V product), stacked [P_hi; P_lo] = 2N rows, MN-major without
       //      swizzle: 8-row x 16-byte core matrices, row blocks 128 B apart,
-      //      8-key groups 32*N B apart; each thread writes its key with 16-byte
-      //      stores into the 8-row blocks of its group's slots (rows past the
+      //      8-key groups 32*N B apart.  Each thread writes its key for its
+      //      group's rows, in units of kAlign rows (16- or 8-byte stores; a
+      //      group's units end before the next group's slots).  Rows past the
       //      group's live ones get zeros; slots no group owns are never read
-      //      back, as O^T column n depends on P row n only).
+      //      back, as O^T column n depends on P row n only.
       {
+        constexpr int U = kAlign;                              // rows per store
+        constexpr int NU = (RG + U - 1) / U;
+        const int nu = kEvenSplit ? NU : (nrows + U - 1) / U;
         const uint32_t pbuf = sP0 + (uint32_t)((i & 1) * KC::kPBufBytes);
-        const uint32_t prow = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16) +
-                              (uint32_t)(slot0 / 8) * 128;
+        const uint32_t pkey = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16);
 #pragma unroll
-        for (int cb = 0; cb < RG8; ++cb) {
-          uint32_t hi[4], lo[4];
+        for (int cb = 0; cb < NU; ++cb) {
+          if (!kEvenSplit && cb >= nu) break;
+          uint32_t hi[U / 2], lo[U / 2];
 #pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const int r0 = cb * 8 + 2 * q2, r1 = r0 + 1;
+          for (int q2 = 0; q2 < U / 2; ++q2) {
+            const int r0 = cb * U + 2 * q2, r1 = r0 + 1;
             float p0 = 0.f, p1 = 0.f;
             if (live(r0)) p0 = exp2f(s[r0] - m_ref[r0]);
             if (live(r1)) p1 = exp2f(s[r1] - m_ref[r1]);
@@ -862,11 +924,18 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             hi[q2] = *reinterpret_cast<const uint32_t*>(&h2);
             lo[q2] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          const uint32_t addr = prow + cb * 128;                 // rows of P_hi
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                       ::"r"(addr), "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"    // rows N.. of P_lo
-                       ::"r"(addr + N * 16), "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
+          const int row = slot0 + cb * U;
+          const uint32_t addr = pkey + (uint32_t)((row >> 3) * 128 + (row & 7) * 2);   // rows of P_hi
+          if constexpr (U == 8) {
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         ::"r"(addr), "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"    // rows N.. of P_lo
+                         ::"r"(addr + N * 16), "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
+          } else {
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(hi[0]), "r"(hi[1]) : "memory");
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};"            // rows N.. of P_lo
+                         ::"r"(addr + N * 16), "r"(lo[0]), "r"(lo[1]) : "memory");
+          }
         }
       }
       // ---- keys no token may see: clear their V rows (stale or poisoned data
@@ -893,7 +962,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         process_o(i, alpha_r);
         RELATTN_TRACE(7, i);
       } else {
-        // both groups are on every tile: take O(i-1) while P.V(i) runs
+        // every group is on every tile: take O(i-1) while P.V(i) runs
         if (last_tile >= 0) {
           process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
           RELATTN_TRACE(7, last_tile);
@@ -915,7 +984,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     //      read); then all softmax threads finish the rows in short loops.
     //      Alternating groups hold the same rows (merged by LSE); column-split
     //      groups hold disjoint rows.
-    bool bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, aborted || failed);
+    bool bad = ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, aborted || failed);
     float* eo = reinterpret_cast<float*>(smem);             // [NG][RG][128]
     float* el = eo + NG * RG * kHeadDim;                    // [NG][RG][128]
     float* em = el + NG * RG * kHeadDim;                    // [NG][RG]
@@ -931,7 +1000,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         for (int r = 0; r < RG; ++r) em[grp * RG + r] = m_ref[r];
       }
     }
-    bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, bad);
+    bad = ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, bad);
     if (!bad) {
       const int et = tid - 64, ew = et >> 5;               // softmax thread / warp index
       // row sums of l: one warp per (group, row)
@@ -940,7 +1009,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         const float v = warp_sum(src[lane] + src[lane + 32] + src[lane + 64] + src[lane + 96]);
         if (lane == 0) es[q] = v;
       }
-      ptx::bar_sync_or(3, kSoftmaxThreads * NG, false);
+      ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, false);
       const int rows = p.B * T * p.Hq;
       // output rows: (token t, head gg) <- entries (group, local row)
       for (int e = et; e < NQ * kHeadDim; e += kSoftmaxThreads * NG) {
@@ -958,8 +1027,15 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             l = fmaf(es[q * RG + n], sc, l);
           }
         } else {
-          const int q = (t >= TA) ? 1 : 0;
-          const int idx = q * RG + (t - q * TA) * G + gg;
+          int q = 0, tq = 0;                        // the group of token t, its first token
+#pragma unroll
+          for (int u = 1; u < NG; ++u) {
+            if (t >= CSp::tok_begin(u)) {
+              q = u;
+              tq = CSp::tok_begin(u);
+            }
+          }
+          const int idx = q * RG + (t - tq) * G + gg;
           m = em[idx];
           o = eo[idx * kHeadDim + d];
           l = es[idx];
