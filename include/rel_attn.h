@@ -18,8 +18,10 @@
  * (learned relative term added to the pre-softmax logits instead of RoPE;
  * GQA with head size 128); "vLLM、Inkling 2 Smallを初日サポート GB200で630
  * tok/s", section "モデルの構成" (48 query / 8 KV heads, sliding window
- * 1,024) and section "vLLMの最適化と性能" (the GQA group's 6 heads packed into
- * one 64-row tile of a decode kernel); "vLLM TML Inkling 지원", section
+ * 1,024; the previous Inkling: 64 / 8 heads on full-attention layers, 64 / 16
+ * with window 512 on sliding ones, so G = 6, 8 and 4) and section
+ * "vLLMの最適化と性能" (the GQA group's 6 heads packed into one 64-row tile
+ * of a decode kernel); "vLLM TML Inkling 지원", section
  * "저지연 컬렉티브 및 커널" (sheared relative bias; num_splits chosen from
  * batch size and KV length).  The pages give no formula: the form and the
  * bucket function above are this library's reading.
@@ -58,7 +60,8 @@ typedef struct rel_attn_shape {
   int batch;             /* B >= 1                                              */
   int q_tokens;          /* T, query tokens per sequence, 1..8 (verify steps)  */
   int num_q_heads;       /* Hq                                                  */
-  int num_kv_heads;      /* Hkv, Hq % Hkv == 0, G = Hq/Hkv == 6, G*T <= 48      */
+  int num_kv_heads;      /* Hkv, Hq % Hkv == 0, G = Hq/Hkv in {4, 6, 8};
+                            T <= 8 for G = 4 and 6, T <= 6 for G = 8          */
   int head_dim;          /* D, must be 128                                      */
   int page_size;         /* P, must be 64                                       */
   int num_pages;         /* pages in the K/V pool                               */
@@ -145,7 +148,8 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
  * either).  The kernels widen the codes to f16 on chip (exact) and run the
  * query through f16 for q.k (exact for |q| in [2^-14, 65504]; smaller
  * magnitudes round to f16 subnormals); the relative term stays bf16.
- * Current limit: shape->q_tokens must be 1 (else REL_ATTN_ERR_INVALID_ARG).
+ * Current limits: shape->q_tokens must be 1 and Hq/Hkv must be 6 (else
+ * REL_ATTN_ERR_INVALID_ARG).
  */
 int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q,
                          const void* k_cache, const void* v_cache,

@@ -26,7 +26,7 @@ struct DeviceInfo {
   bool probed = false;
   bool sm100 = false;
   int sm_count = 0;
-  bool attr_set[kMaxQTokens] = {};
+  bool attr_set[3][kMaxQTokens] = {};     // [G = 4, 6, 8][T - 1]
   bool attr_fp8 = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -49,16 +49,9 @@ bool encode_fn_ready() {
   return g_encode != nullptr;
 }
 
-// Group width N (GQA group x query tokens, padded to the MMA N step of 16).
-// The 16-wide instance serves one token (6 rows); 32 and 48 hold one row block
-// per softmax group (blocks 8-aligned, or 4-aligned where 8 does not fit).
-int group_width(int G, int T) {
-  const int nq = G * T;
-  if (nq <= 6) return 16;
-  if (nq <= 24) return 32;     // two groups' rows, 8-aligned blocks, in 32 slots
-  if (nq <= 48) return 48;
-  return 0;
-}
+// GQA group sizes with kernel instances: 48/8 heads (Inkling 2 Small, every
+// layer) and the 64/8 full / 64/16 sliding layers of the previous Inkling.
+bool group_supported(int G) { return G == 4 || G == 6 || G == 8; }
 
 int validate_shape(const rel_attn_shape* s) {
   if (!s) return REL_ATTN_ERR_INVALID_ARG;
@@ -66,8 +59,8 @@ int validate_shape(const rel_attn_shape* s) {
   if (s->q_tokens < 1 || s->q_tokens > kMaxQTokens) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_kv_heads < 1 || s->num_kv_heads > 65535) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_q_heads < 1 || s->num_q_heads % s->num_kv_heads) return REL_ATTN_ERR_INVALID_ARG;
-  if (s->num_q_heads / s->num_kv_heads != 6) return REL_ATTN_ERR_INVALID_ARG;
-  if (group_width(6, s->q_tokens) == 0) return REL_ATTN_ERR_INVALID_ARG;
+  const int G = s->num_q_heads / s->num_kv_heads;
+  if (!group_supported(G) || group_width_for(G, s->q_tokens) == 0) return REL_ATTN_ERR_INVALID_ARG;
   if (s->head_dim != kHeadDim || s->page_size != kPage) return REL_ATTN_ERR_INVALID_ARG;
   if (s->num_pages < 1 || s->max_pages_per_seq < 1) return REL_ATTN_ERR_INVALID_ARG;
   if ((long long)s->num_pages * s->num_kv_heads * kPage >= (1ll << 31)) return REL_ATTN_ERR_INVALID_ARG;
@@ -258,22 +251,42 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
   return true;
 }
 
-template <int T>
+template <int G, int T>
 int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
-  constexpr int N = (T == 1) ? 16 : (T <= 4 ? 32 : 48);              // group width, as group_width()
-  constexpr int NG = softmax_groups(T);
-  constexpr int slot = T - 1;
-  using KC = KernelConfig<N, NG>;
-  auto kern = rel_attn_partial_kernel<N, 6, NG, T>;
-  constexpr int smem = KC::kAllocBytes;
-  if (!di.attr_set[slot]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return REL_ATTN_ERR_CUDA;
-    di.attr_set[slot] = true;
+  constexpr int N = group_width_for(G, T);
+  if constexpr (N == 0) {
+    return REL_ATTN_ERR_INVALID_ARG;                  // no instance for this shape
+  } else {
+    constexpr int NG = softmax_groups(G, T);
+    using KC = KernelConfig<N, NG, G>;
+    auto kern = rel_attn_partial_kernel<N, G, NG, T>;
+    constexpr int smem = KC::kAllocBytes;
+    bool& attr = di.attr_set[G / 2 - 2][T - 1];
+    if (!attr) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return REL_ATTN_ERR_CUDA;
+      attr = true;
+    }
+    dim3 grid(S, Hkv, B);
+    kern<<<grid, KC::kThreads, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
   }
-  dim3 grid(S, Hkv, B);
-  kern<<<grid, KC::kThreads, smem, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
+}
+
+template <int G>
+int launch_partial_group(const DecodeParams& prm, int T, int S, int B, int Hkv, cudaStream_t st,
+                         DeviceInfo& di) {
+  switch (T) {
+    case 1: return launch_partial<G, 1>(prm, S, B, Hkv, st, di);
+    case 2: return launch_partial<G, 2>(prm, S, B, Hkv, st, di);
+    case 3: return launch_partial<G, 3>(prm, S, B, Hkv, st, di);
+    case 4: return launch_partial<G, 4>(prm, S, B, Hkv, st, di);
+    case 5: return launch_partial<G, 5>(prm, S, B, Hkv, st, di);
+    case 6: return launch_partial<G, 6>(prm, S, B, Hkv, st, di);
+    case 7: return launch_partial<G, 7>(prm, S, B, Hkv, st, di);
+    case 8: return launch_partial<G, 8>(prm, S, B, Hkv, st, di);
+    default: return REL_ATTN_ERR_INVALID_ARG;
+  }
 }
 
 }  // namespace
@@ -377,7 +390,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
   if (kv_e4m3) {
-    if (shape->q_tokens != 1 || !k_scale || !v_scale ||
+    if (shape->q_tokens != 1 || shape->num_q_heads != 6 * shape->num_kv_heads || !k_scale || !v_scale ||
         (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))
       return REL_ATTN_ERR_INVALID_ARG;
   }
@@ -405,7 +418,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
   if (!cached_map(&prm->tmap_k, kv_e4m3 ? 4 : 0, k_cache, kv_rows, 0) ||
       !cached_map(&prm->tmap_v, kv_e4m3 ? 5 : 1, v_cache, kv_rows, 0) ||
-      !cached_map(&prm->tmap_r, group_width(6, T) == 16 ? 3 : 2, rel_table,
+      !cached_map(&prm->tmap_r, group_width_for(Hq / Hkv, T) == 16 ? 3 : 2, rel_table,
                   (uint64_t)shape->num_buckets, (uint64_t)Hkv))
     return REL_ATTN_ERR_CUDA;
   prm->q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -435,16 +448,11 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
 
 int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
                        DeviceInfo& di) {
-  const int B = shape->batch, Hkv = shape->num_kv_heads;
-  switch (shape->q_tokens) {
-    case 1: return launch_partial<1>(prm, S, B, Hkv, st, di);
-    case 2: return launch_partial<2>(prm, S, B, Hkv, st, di);
-    case 3: return launch_partial<3>(prm, S, B, Hkv, st, di);
-    case 4: return launch_partial<4>(prm, S, B, Hkv, st, di);
-    case 5: return launch_partial<5>(prm, S, B, Hkv, st, di);
-    case 6: return launch_partial<6>(prm, S, B, Hkv, st, di);
-    case 7: return launch_partial<7>(prm, S, B, Hkv, st, di);
-    case 8: return launch_partial<8>(prm, S, B, Hkv, st, di);
+  const int B = shape->batch, Hkv = shape->num_kv_heads, T = shape->q_tokens;
+  switch (shape->num_q_heads / Hkv) {
+    case 4: return launch_partial_group<4>(prm, T, S, B, Hkv, st, di);
+    case 6: return launch_partial_group<6>(prm, T, S, B, Hkv, st, di);
+    case 8: return launch_partial_group<8>(prm, T, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }

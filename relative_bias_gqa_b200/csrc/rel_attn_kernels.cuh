@@ -64,11 +64,13 @@ constexpr int kSoftmaxThreads = 128;           // one softmax group
 // named barriers: 1 .. NG one per softmax group, then these two
 constexpr int kBarSoftmaxAll = 5;              // every softmax thread (epilogue)
 constexpr int kBarSetup = 6;                   // every warp but the producer (prologue)
-// Softmax groups of the instance for T query tokens: two for up to five
-// tokens, four beyond (each group then carries at most 12 rows of S^T, so a
-// thread's per-tile work halves and every SM sub-partition runs four softmax
-// warps to hide each other's latencies).
-__host__ __device__ constexpr int softmax_groups(int T) { return T >= 6 ? 4 : 2; }
+// Softmax groups of the instance for G heads per KV head and T query tokens:
+// four from six tokens on where each group then carries at most 12 rows of
+// S^T (a thread's per-tile work halves and every SM sub-partition runs four
+// softmax warps to hide each other's latencies), else two.
+__host__ __device__ constexpr int softmax_groups(int G, int T) {
+  return (T >= 6 && (T + 3) / 4 * G <= 12) ? 4 : 2;
+}
 constexpr int kVSlotBytes = 32768;             // V tile: 128 keys x 128 dims bf16
 constexpr int kHalfTileBytes = 16384;          // 128 rows x 128 B (one 64-dim half)
 constexpr int kPageHalfBytes = 8192;           // 64 rows x 128 B
@@ -109,11 +111,12 @@ struct alignas(64) DecodeParams {
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 // Compile-time configuration of one kernel instance: N = padded group width
-// (G heads x T tokens rounded up to the MMA N step), NG = softmax groups.
+// (G heads x T tokens rounded up to the MMA N step), NG = softmax groups,
+// G = query heads per KV head.
 // K tiles and relative-row chunks share one ring of slots (each slot is
 // released as soon as its MMA has read it); V tiles have their own, deeper
 // ring (a V slot is held until the P.V product of its tile).
-template <int N, int NG>
+template <int N, int NG, int G>
 struct KernelConfig {
   // N = 16 (one token): the softmax groups alternate tiles, each with all the
   // rows.  N = 32 / 48 (2..8 tokens): every group takes every tile, each with
@@ -134,8 +137,8 @@ struct KernelConfig {
   static constexpr int kVSlots = (N == 16) ? 4 : (N == 32 ? 3 : 2);
   static constexpr int kVLag = 0;                               // V issued this many tiles after K
   // Relative-table gather stride: odd for conflict-free gathers.  The N = 16
-  // instance serves at most 6 live rows.
-  static constexpr int kYStride = (N == 16) ? 7 : N + 1;
+  // instance serves G live rows (one token).
+  static constexpr int kYStride = (N == 16) ? (G % 2 == 0 ? G + 1 : G + 2) : N + 1;
   static constexpr int kOperandBytes = 2 * N * 128;            // N rows x 128 dims, two 64-dim halves
   static constexpr int kPBufBytes = 2 * kOperandBytes;         // [P_hi; P_lo]: 128 keys x 2N rows
   static constexpr int kYBytes = align_up(kRows * kYStride * 4, 16);
@@ -171,19 +174,43 @@ struct KernelConfig {
 // slot(q, A) on, slots packed with alignment A = 8 where that fits in N, else
 // 4 (a 4-aligned group reads its tensor-memory columns from the 8-aligned
 // column below and shifts by four).
+__host__ __device__ constexpr int cs_tok_begin(int T, int NG, int q) { return q * T / NG; }
+__host__ __device__ constexpr int cs_rows(int T, int G, int NG, int q) {
+  return (cs_tok_begin(T, NG, q + 1) - cs_tok_begin(T, NG, q)) * G;
+}
+__host__ __device__ constexpr int cs_slot(int T, int G, int NG, int q, int a) {
+  int s = 0;
+  for (int u = 0; u < q; ++u) s = align_up(s + cs_rows(T, G, NG, u), a);
+  return s;
+}
+__host__ __device__ constexpr int cs_end(int T, int G, int NG, int a) {
+  return align_up(cs_slot(T, G, NG, NG - 1, a) + cs_rows(T, G, NG, NG - 1), a);
+}
+
 template <int T, int G, int NG>
 struct ColSplit {
-  __host__ __device__ static constexpr int tok_begin(int q) { return q * T / NG; }
-  __host__ __device__ static constexpr int rows(int q) { return (tok_begin(q + 1) - tok_begin(q)) * G; }
-  __host__ __device__ static constexpr int slot(int q, int a) {
-    int s = 0;
-    for (int u = 0; u < q; ++u) s = align_up(s + rows(u), a);
-    return s;
-  }
-  __host__ __device__ static constexpr int end(int a) { return align_up(slot(NG - 1, a) + rows(NG - 1), a); }
+  __host__ __device__ static constexpr int tok_begin(int q) { return cs_tok_begin(T, NG, q); }
+  __host__ __device__ static constexpr int rows(int q) { return cs_rows(T, G, NG, q); }
+  __host__ __device__ static constexpr int slot(int q, int a) { return cs_slot(T, G, NG, q, a); }
+  __host__ __device__ static constexpr int end(int a) { return cs_end(T, G, NG, a); }
   __host__ __device__ static constexpr int align(int n) { return end(8) <= n ? 8 : 4; }
   static constexpr int kMaxRows = (T + NG - 1) / NG * G;
 };
+
+// Group width N of the instance for G heads per KV head and T tokens (0: not
+// supported): 16 for one token (the alternating-group instance, G <= 8);
+// otherwise the smaller of 32 and 48 whose query slots hold every softmax
+// group's row block 8-aligned, else the smaller one that holds them 4-aligned.
+__host__ __device__ constexpr int group_width_for(int G, int T) {
+  if (G < 1 || G > 8 || T < 1 || T > 8) return 0;
+  if (T == 1) return 16;
+  const int NG = softmax_groups(G, T);
+  if (cs_end(T, G, NG, 8) <= 32) return 32;
+  if (cs_end(T, G, NG, 8) <= 48) return 48;
+  if (cs_end(T, G, NG, 4) <= 32) return 32;
+  if (cs_end(T, G, NG, 4) <= 48) return 48;
+  return 0;
+}
 
 // Per-CTA geometry shared by the three roles.
 struct SplitGeom {
@@ -354,9 +381,9 @@ __device__ void fill_rows(const DecodeParams& p, int b, int h, int s, float o_va
 // T (query tokens) is a template parameter: every per-row loop below runs
 // over the NQ = T*G live rows only, fully unrolled.
 template <int N, int G, int NG, int T>
-__global__ void __launch_bounds__(KernelConfig<N, NG>::kThreads, 1)
+__global__ void __launch_bounds__(KernelConfig<N, NG, G>::kThreads, 1)
 rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
-  using KC = KernelConfig<N, NG>;
+  using KC = KernelConfig<N, NG, G>;
   constexpr int KS = KC::kKSlots;
   constexpr int VS = KC::kVSlots;
   constexpr int ROWS = KC::kRows;
@@ -380,7 +407,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int RG8 = (RG + 7) / 8;
   constexpr int RGL8 = (kAlign == 8) ? RG8 : (RG + 4 + 7) / 8;   // 8-column loads per row block
   constexpr bool kEvenSplit = KC::kAlt || T % NG == 0;
-  static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(T) && CSp::end(kAlign) <= N &&
+  static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(G, T) && CSp::end(kAlign) <= N &&
                                                    RG <= KC::kGR), "group width");
   RELATTN_TRACE(16, 0);
 

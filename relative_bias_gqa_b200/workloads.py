@@ -6,7 +6,9 @@ arithmetic, so both the CUDA path and the CPU oracle may be fed from it.
 Shapes follow the Inkling model descriptions:
   * "vLLM、Inkling 2 Smallを初日サポート GB200で630 tok/s", section
     "モデルの構成" (table rows "Heads" and "Sliding window"): 48 query / 8 KV
-    heads on every layer, sliding window 1,024.
+    heads on every layer, sliding window 1,024; the previous Inkling's
+    full-attention layers 64 query / 8 KV heads, its sliding layers 64 / 16
+    with window 512.
   * "vLLM TML Inkling 지원", section "TML Inkling 모델 아키텍처": GQA with head
     size 128, context up to 1M tokens, up to 9 tokens per speculative step.
   * same page, section "Sconv 캐시 및 TP 샤딩": the KV cache is held by a
@@ -146,7 +148,7 @@ def batched_lengths(batch: int = 32, lo: int = 16384, hi: int = 131072,
     return torch.randint(lo, hi + 1, (batch,), generator=g).tolist()
 
 
-# The five named workloads (shapes from the Inkling model descriptions).
+# The named workloads (shapes from the Inkling model descriptions).
 WORKLOADS = {
     # tiny oracle-scale case: 6 query heads / 1 KV head, 2,048 keys, contiguous cache
     "tiny_2k": dict(seq_lens=[2048], num_q_heads=6, num_kv_heads=1, window=0,
@@ -160,6 +162,12 @@ WORKLOADS = {
                            num_buckets=1280),
     # 32 sequences with lengths uniform in [16,384, 131,072], one shared pool
     "batched_32": dict(seq_lens=None, window=0, num_buckets=1280),
+    # the previous Inkling's layers over a 100,000-token context: full
+    # attention with 64 query / 8 KV heads, sliding window 512 with 64 / 16
+    "v1_full_100k": dict(seq_lens=[100_000], window=0, num_buckets=1280,
+                         num_q_heads=64, num_kv_heads=8),
+    "v1_sliding_100k": dict(seq_lens=[100_000], window=512, num_buckets=1024,
+                            num_q_heads=64, num_kv_heads=16),
 }
 
 

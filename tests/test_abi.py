@@ -71,7 +71,9 @@ def test_host_bucket_every_distance_nb1280(ra):
 
 BAD = [
     dict(q_tokens=0), dict(q_tokens=9), dict(head_dim=64), dict(page_size=16),
-    dict(num_q_heads=47), dict(num_q_heads=64), dict(num_kv_heads=0), dict(batch=0),
+    dict(num_q_heads=47), dict(num_q_heads=24), dict(num_q_heads=40), dict(num_q_heads=56),
+    dict(num_q_heads=80), dict(num_q_heads=64, q_tokens=7), dict(num_q_heads=64, q_tokens=8),
+    dict(num_kv_heads=0), dict(batch=0),
     dict(num_buckets=0), dict(num_buckets=1024 + 513), dict(num_pages=0),
     dict(max_pages_per_seq=0), dict(out_fp32=2), dict(max_seq_len=-1),
     dict(num_pages=1 << 23),
@@ -86,6 +88,29 @@ def test_invalid_shape_rejected_before_any_cuda_call(ra, kw):
                                 fake, None, fake, 1 << 30, None)
     assert rc == ra.REL_ATTN_ERR_INVALID_ARG
     assert ra.rel_attn_workspace_bytes(s, 4) == 0
+
+
+# Group sizes with instances: 48/8 (G = 6), the previous Inkling's 64/8 full
+# (G = 8, up to 6 tokens: 8 x 6 rows fill the 48 query slots) and 64/16
+# sliding (G = 4) layers.
+GOOD = [dict(num_q_heads=48, num_kv_heads=8, q_tokens=t) for t in range(1, 9)] + \
+       [dict(num_q_heads=64, num_kv_heads=8, q_tokens=t) for t in range(1, 7)] + \
+       [dict(num_q_heads=64, num_kv_heads=16, q_tokens=t) for t in range(1, 9)]
+
+
+@pytest.mark.parametrize("kw", GOOD, ids=[f"{k['num_q_heads']}/{k['num_kv_heads']}-T{k['q_tokens']}" for k in GOOD])
+def test_supported_group_shapes(ra, kw):
+    s = shape(ra, **kw)
+    rows = kw["q_tokens"] * kw["num_q_heads"]
+    assert ra.rel_attn_workspace_bytes(s, 3) == 256 + (3 * rows * 4 + 255) // 256 * 256 + 3 * rows * 128 * 4
+
+
+def test_e4m3_only_for_48_over_8(ra):
+    s = shape(ra, num_q_heads=64, num_kv_heads=8)
+    fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+    rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
+                                     fake, 0, 1, fake, None, fake, 1 << 30, None)
+    assert rc == ra.REL_ATTN_ERR_INVALID_ARG
 
 
 def test_invalid_pointers_and_splits(ra):

@@ -287,3 +287,59 @@ def test_status_clean_after_normal_call(ra):
     ws = Workspace.for_shape(shape, 0, "cuda")
     run_gpu(ra, case, 0, workspace=ws)
     assert ws.read_status() == ra.REL_ATTN_OK
+
+
+# ------------------------------------------- other GQA group sizes (G = 4, 8)
+# The previous Inkling's layers: 64 query / 8 KV heads on full attention
+# (G = 8, up to 6 tokens) and 64 / 16 on sliding-window layers (G = 4, window
+# 512).  Each (G, T) pair has its own kernel instance.
+def small_g(L, G, T=1, window=0, NB=1280, seed=0, Hkv=2, lens=None, **kw):
+    lens = lens if lens is not None else [L]
+    return W.make_case(seq_lens=lens, q_tokens=T, num_q_heads=G * Hkv, num_kv_heads=Hkv,
+                       window=window, num_buckets=NB, seed=seed, extra_pages=2, **kw).to("cuda")
+
+
+GROUP_CASES = (
+    [dict(G=8, T=t, L=L) for t in range(1, 7) for L in (t, 129, 2100)] +
+    [dict(G=4, T=t, L=L) for t in range(1, 9) for L in (t, 129, 2100)] +
+    [dict(G=8, T=1, L=3001, window=1024, NB=1024), dict(G=8, T=6, L=3000, window=100),
+     dict(G=4, T=1, L=3001, window=512, NB=1024), dict(G=4, T=8, L=2500, window=512, NB=1024),
+     dict(G=4, T=5, L=1500, window=64), dict(G=8, T=3, L=5000, seed=3),
+     dict(G=8, T=5, L=3000, NB=200, exact_buckets=16, max_distance=100000),
+     dict(G=4, T=7, L=6000, NB=364, exact_buckets=64, max_distance=5000)]
+)
+
+
+@pytest.mark.parametrize("kw", GROUP_CASES, ids=[str(k) for k in GROUP_CASES])
+def test_other_group_sizes(ra, kw):
+    case = small_g(**kw)
+    ref = run_oracle(case)
+    for splits in (1, 3, 0):
+        check(*run_gpu(ra, case, splits), *ref)
+
+
+@pytest.mark.parametrize("G,T", [(8, 2), (8, 6), (4, 3), (4, 8)])
+def test_other_group_sizes_batched(ra, G, T):
+    case = small_g(0, G, T=T, Hkv=3, lens=[T, 64, 65 + T, 300, 1111, 2049, 129, T + 1])
+    ref = run_oracle(case)
+    for splits in (1, 2, 5, 0):
+        check(*run_gpu(ra, case, splits), *ref)
+
+
+@pytest.mark.parametrize("name", ["v1_full_100k", "v1_sliding_100k"])
+def test_previous_model_layers_100k(ra, name):
+    case = W.make_workload(name, seed=0, device="cuda")
+    ref = run_oracle(case)
+    for splits in (1, 7, 0):
+        check(*run_gpu(ra, case, splits), *ref)
+
+
+@pytest.mark.parametrize("G,T", [(8, 6), (4, 8)])
+def test_other_group_sizes_verify_256k(ra, G, T):
+    """Full-size verify with the G = 8 / G = 4 instances (one KV head keeps the
+    oracle fast; the sequence still spans every split)."""
+    case = W.make_case(seq_lens=[262_144], q_tokens=T, num_q_heads=G, num_kv_heads=1,
+                       window=0, num_buckets=1280, seed=0).to("cuda")
+    ref = run_oracle(case)
+    for splits in (1, 18, 0):
+        check(*run_gpu(ra, case, splits), *ref)
