@@ -276,6 +276,39 @@ def test_gqa_head_mapping():
         assert np.abs(out[0, :, hq] - (hq // 2 + 1)).max() <= 1e-12
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (16, 2), (16, 4)])
+def test_gqa_head_mapping_other_group_sizes(Hq, Hkv):
+    # G = 4 and 8 (the previous Inkling's 64/16 and 64/8 layers, scaled down)
+    case = small_case(L=70, T=3, Hq=Hq, Hkv=Hkv, D=8, P=8)
+    for h in range(Hkv):
+        case.v_cache[:, h] = float(h + 1)
+    out, _ = run_ref(case)
+    G = Hq // Hkv
+    for hq in range(Hq):
+        assert np.abs(out[0, :, hq] - (hq // G + 1)).max() <= 1e-12
+
+
+@pytest.mark.parametrize("Hq,Hkv,T,window", [(16, 2, 6, 0), (8, 2, 8, 7), (16, 4, 1, 0)])
+def test_zero_rel_is_sdpa_other_group_sizes(Hq, Hkv, T, window):
+    case = small_case(L=120, T=T, Hq=Hq, Hkv=Hkv, D=16, P=8, window=window)
+    case.rel_table.zero_()
+    out, lse = run_ref(case)
+    L, G = 120, Hq // Hkv
+    pages = case.block_table[0].long()
+    j = torch.arange(L)
+    k = case.k_cache.double()[pages[j // 8], :, j % 8].repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    v = case.v_cache.double()[pages[j // 8], :, j % 8].repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    q = case.q.double()[0].permute(1, 0, 2)[None]
+    p = torch.arange(L - T, L)[:, None]
+    mask = (j[None] <= p)
+    if window > 0:
+        mask &= (p - j[None]) <= window - 1
+    sd = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+    assert np.abs(out[0] - sd[0].permute(1, 0, 2).numpy()).max() <= 1e-12
+    logits = ((q @ k.transpose(-1, -2)) / math.sqrt(16)).masked_fill(~mask, float("-inf"))
+    assert np.abs(lse[0] - torch.logsumexp(logits, dim=-1)[0].permute(1, 0).numpy()).max() <= 1e-12
+
+
 # ------------------------------------------------- planted mistakes are caught
 def _pins_fail(monkeypatch, name, bad):
     monkeypatch.setattr(ref, name, bad)
