@@ -453,7 +453,7 @@ def run_reference(args, rank, world):
     t0 = time.perf_counter()
     one(n)
     dt = time.perf_counter() - t0
-    n = int(max(1024, min(len(keys), n * budget / max(dt, 1e-6))))
+    n = int(min(len(keys), max(1024, n * budget / max(dt, 1e-6))))   # never past the visible keys
     for _ in range(args.warmup):
         one(n)
     t0 = time.perf_counter()

@@ -75,3 +75,14 @@ def test_two_ranks_take_the_slowest_device_time():
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(7.25, 1, torch.device("cpu")) == 7.25
     assert bench.whole_job_gbs(1, 10, 1000, 1.0) == pytest.approx(10 * 1000 / 1e-3 / 1e9)
+
+
+def test_reference_arm_sample_stays_inside_the_window():
+    """With a 512-key window the oracle sample holds at most the visible keys
+    (the bytes it reports are the bytes it read)."""
+    import re
+    ref = bench.run_reference(types.SimpleNamespace(workload="v1_sliding_100k", seed=0, steps=1,
+                                                    warmup=0), 0, 1)
+    n = int(re.search(r"the last (\d+) visible keys", ref["cpu_baseline"]["sample"]).group(1))
+    assert 0 < n <= 512
+    assert ref["value"] == ref["cpu_baseline"]["value"] > 0
