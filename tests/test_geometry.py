@@ -1,0 +1,100 @@
+"""Row-block geometry of the partial kernel's instances, read from the kernel
+header itself: a host program compiled against rel_attn_kernels.cuh prints,
+for every G (heads per KV head) and T (query tokens), the group width N, the
+softmax group count and each group's tokens and query slots; the checks below
+are the layout rules the kernel relies on (no GPU needed).
+"""
+
+import os
+import subprocess
+
+import pytest
+
+from relative_bias_gqa_b200 import build as B
+
+PROGRAM = r"""
+#include <cstdio>
+#include "rel_attn_kernels.cuh"
+using namespace relattn;
+int main() {
+  for (int G = 1; G <= 8; ++G) {
+    for (int T = 1; T <= 8; ++T) {
+      const int N = group_width_for(G, T), NG = softmax_groups(G, T);
+      const int A = (T == 1) ? 8 : (cs_end(T, G, NG, 8) <= N ? 8 : 4);
+      std::printf("%d %d %d %d %d", G, T, N, NG, A);
+      for (int q = 0; q < NG; ++q)
+        std::printf(" %d:%d:%d", cs_tok_begin(T, NG, q), cs_slot(T, G, NG, q, A), cs_rows(T, G, NG, q));
+      std::printf("\n");
+    }
+  }
+  return 0;
+}
+"""
+
+
+@pytest.fixture(scope="module")
+def table(tmp_path_factory):
+    d = tmp_path_factory.mktemp("geom")
+    src = d / "geom.cu"
+    src.write_text(PROGRAM)
+    exe = d / "geom"
+    cmd = [B.find_nvcc(), "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+           "-I", B.INCLUDE, "-I", B.CSRC, "-o", str(exe), str(src)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    rows = {}
+    for line in out.splitlines():
+        f = line.split()
+        G, T, N, NG, A = map(int, f[:5])
+        groups = [tuple(map(int, g.split(":"))) for g in f[5:]]
+        rows[(G, T)] = (N, NG, A, groups)
+    return rows
+
+
+SUPPORTED = [(6, t) for t in range(1, 9)] + [(8, t) for t in range(1, 7)] + [(4, t) for t in range(1, 9)]
+
+
+def test_supported_shapes_have_instances(table):
+    for G, T in SUPPORTED:
+        assert table[(G, T)][0] in (16, 32, 48), (G, T)
+    assert table[(8, 7)][0] == 0 and table[(8, 8)][0] == 0       # 56 / 64 rows > 48 slots
+
+
+def test_inkling2_instances(table):
+    # 48/8 heads: N and group counts of the measured instances
+    assert [table[(6, t)][0] for t in range(1, 9)] == [16, 32, 32, 32, 48, 48, 48, 48]
+    assert [table[(6, t)][1] for t in range(1, 9)] == [2, 2, 2, 2, 2, 4, 4, 4]
+    assert [table[(6, t)][2] for t in range(6, 9)] == [8, 4, 4]       # 4-aligned at T = 7, 8
+
+
+@pytest.mark.parametrize("G,T", [k for k in SUPPORTED if k[1] >= 2])
+def test_column_split_layout(table, G, T):
+    N, NG, A, groups = table[(G, T)]
+    assert len(groups) == NG
+    # tokens: a partition of [0, T) in order, every group non-empty
+    starts = [g[0] for g in groups] + [T]
+    assert starts[0] == 0 and all(starts[q] < starts[q + 1] for q in range(NG))
+    for q, (tb, slot, rows) in enumerate(groups):
+        assert rows == (starts[q + 1] - tb) * G
+        assert slot % A == 0
+        # the group's P units (A rows each) end before the next group's slots
+        end = slot + -(-rows // A) * A
+        nxt = groups[q + 1][1] if q + 1 < NG else N
+        assert end <= nxt <= N
+        # at most the per-group row capacity of the instance
+        assert rows <= N // NG
+        # tensor-memory loads: RG = the instance's row capacity per group,
+        # read as 8-column loads from the slot (A = 8) or from the 8-aligned
+        # column below it, RG + 4 columns (A = 4); they must end inside the
+        # group's N-column buffer (S, each O half, X0 and X1 are N wide, and
+        # X1 is the last block of the allocation)
+        RG = -(-T // NG) * G
+        base, cols = (slot, -(-RG // 8) * 8) if A == 8 else (slot & ~7, -(-(RG + 4) // 8) * 8)
+        assert base + cols <= N, (q, base, cols)
+
+
+@pytest.mark.parametrize("G", [4, 6, 8])
+def test_one_token_instance(table, G):
+    N, NG, A, groups = table[(G, 1)]
+    assert N == 16 and NG == 2 and G <= N
