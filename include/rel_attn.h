@@ -36,6 +36,10 @@
  *   - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  The caller synchronises.
  *   - One workspace must not be used by two calls that run concurrently.
+ *   - Host threads: the library keeps process-wide caches (per-device
+ *     attributes, encoded tensor maps, bucket-edge tables) that are not
+ *     locked.  Issue calls from one host thread at a time (any number of
+ *     streams); callers with several host threads serialise the calls.
  */
 #ifndef REL_ATTN_H
 #define REL_ATTN_H
