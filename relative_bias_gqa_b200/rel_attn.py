@@ -181,6 +181,8 @@ def rel_attn_decode(q, k_cache, v_cache, block_table, seq_lens, rel_table,
     q bf16 [B, T, Hq, D]; k_cache / v_cache bf16 [num_pages, Hkv, P, D];
     block_table int32 [B, max_pages]; seq_lens int32 [B]; rel_table bf16
     [Hkv, NB, D] -- all contiguous CUDA tensors.  Returns (out, lse).
+    Supported: D = 128, P = 64, Hq / Hkv in {4, 6, 8} with T <= 8 (T <= 6
+    for 8); other shapes raise RelAttnError (REL_ATTN_ERR_INVALID_ARG).
     """
     for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
                         ("v_cache", v_cache, torch.bfloat16), ("rel_table", rel_table, torch.bfloat16),
