@@ -139,6 +139,11 @@ def test_split_heuristic_values(ra):
     assert 1 <= v <= 4
     for sm in (1, 7, 148, 1000):
         assert 1 <= ra.rel_attn_choose_splits(shape(ra), 0, sm) <= 256
+    # the previous Inkling's layers: 64/8 full behaves like 48/8 (8 KV heads);
+    # 64/16 sliding has 16 units per split and a 512-key window (5 tiles)
+    assert ra.rel_attn_choose_splits(shape(ra, num_q_heads=64), 0, 148) == 18
+    assert ra.rel_attn_choose_splits(shape(ra, num_q_heads=64, num_kv_heads=16), 0, 148) == 9
+    assert ra.rel_attn_choose_splits(shape(ra, num_q_heads=64, num_kv_heads=16), 512, 148) == 5
 
 
 def test_workspace_bytes(ra):
