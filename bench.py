@@ -170,29 +170,51 @@ def load_traffic(src_hash, workload):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_throughput(case, seconds: float, kv_heads: int = 1):
-    """The fp64 oracle, as it stands, on KV head 0 of the workload (its G
-    query heads over the whole visible context), repeated for ~`seconds`."""
-    import numpy as np
-    import oracle
+def head0_subcase(case, kv=None):
+    """Sequence 0, KV head 0 of the workload as a compact host problem: its
+    G query heads, the pages it walks (renumbered 0..n-1), relative table 0.
+    ``kv`` = (k_codes, v_codes, k_scale, v_scale) for an E4M3 cache."""
     G = case.num_q_heads // case.num_kv_heads
-    idx = case.block_table[0].long()
     L = int(case.seq_lens[0])
     n_pages = math.ceil(L / case.page_size)
-    pages = idx[:n_pages]
-    sub_k = case.k_cache[pages][:, :kv_heads].cpu()
-    sub_v = case.v_cache[pages][:, :kv_heads].cpu()
-    bt = torch_arange_row(n_pages)
-    q = case.q[:1, :, :G * kv_heads].cpu()
-    rel = case.rel_table[:kv_heads].cpu()
-    sl = case.seq_lens[:1].cpu()
+    pages = case.block_table[0, :n_pages].long()
+    sub = dict(q=case.q[:1, :, :G].cpu(), bt=torch_arange_row(n_pages),
+               sl=case.seq_lens[:1].cpu(), rel=case.rel_table[:1].cpu())
+    if kv is None:
+        sub["k"] = case.k_cache[pages][:, :1].cpu()
+        sub["v"] = case.v_cache[pages][:, :1].cpu()
+    else:
+        kc, vc, ks, vs = kv
+        sub["k"] = kc[pages][:, :1].cpu()
+        sub["v"] = vc[pages][:, :1].cpu()
+        sub["ks"], sub["vs"] = ks[:1].cpu(), vs[:1].cpu()
+    return sub
+
+
+def oracle_head0(case, sub):
+    """The fp64 oracle, as it stands, on the head-0 sub-problem."""
+    import oracle
+    if "ks" in sub:
+        return oracle.rel_attn_decode_fp8kv_ref(sub["q"], sub["k"], sub["v"], sub["ks"], sub["vs"],
+                                                sub["bt"], sub["sl"], sub["rel"], case.window)
+    return oracle.rel_attn_decode_ref(sub["q"], sub["k"], sub["v"], sub["bt"], sub["sl"],
+                                      sub["rel"], case.window)
+
+
+def oracle_throughput(case, sub, seconds: float):
+    """The oracle on KV head 0 of sequence 0 (its G query heads over the
+    whole visible context), repeated for ~`seconds`; returns the baseline
+    record and the last result (for the parity sample)."""
+    L = int(case.seq_lens[0])
     W = case.window
     lo = max(0, L - case.q_tokens - W + 1) if W > 0 else 0
-    nbytes = (L - lo) * kv_heads * 128 * 4
+    elem = 1 if "ks" in sub else 2
+    nbytes = (L - lo) * 128 * 2 * elem
+    G = case.num_q_heads // case.num_kv_heads
     t0 = time.perf_counter()
     calls = 0
     while True:
-        oracle.rel_attn_decode_ref(q, sub_k, sub_v, bt, sl, rel, W)
+        res = oracle_head0(case, sub)
         calls += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -200,9 +222,10 @@ def oracle_throughput(case, seconds: float, kv_heads: int = 1):
     cores = len(os.sched_getaffinity(0))
     return {"value": calls * nbytes / el / 1e9, "unit": "GB/s", "cores": cores,
             "kind": "oracle",
-            "sample": (f"KV head 0 of {case.name} ({G} query heads, {L - lo} visible keys), "
-                       f"{calls} calls in {el:.1f} s; numpy fp64 with up to {cores} BLAS threads"),
-            "seconds": el}
+            "sample": (f"KV head 0 of sequence 0 of {case.name} ({G} query heads x "
+                       f"{case.q_tokens} token(s), {L - lo} visible keys), {calls} calls in "
+                       f"{el:.1f} s; numpy fp64 with up to {cores} BLAS threads"),
+            "seconds": el}, res
 
 
 def torch_arange_row(n):
@@ -241,6 +264,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     case = workloads.make_workload(args.workload, seed=args.seed + rank, device=dev)
     e4m3 = args.kv_dtype == "e4m3"
+    kc = vc = ks = vs = None
     if e4m3:
         kc, vc, ks, vs = workloads.to_e4m3(case)
         kv_args = dict(k_cache=kc, v_cache=vc, scales=dict(k_scale=ks, v_scale=vs))
@@ -354,6 +378,31 @@ def run_ours(args, rank, world, local_rank):
     h2d = h_in.numel()
     d2h = h_res.numel()
 
+    # Parity sample on the timed inputs: the same call with an fp32 output
+    # (the tolerance's reference point) against the oracle's rows for KV head
+    # 0 of sequence 0; outside every timed region.
+    parity = None
+    cpu = None
+    if rank == 0:
+        G = case.num_q_heads // case.num_kv_heads
+        prep32 = rel_attn.Prepared(case.q, kv_args["k_cache"], kv_args["v_cache"], case.block_table,
+                                   case.seq_lens, case.rel_table, case.window, S,
+                                   max_seq_len=case.max_seq_len, out_fp32=True, **kv_args["scales"])
+        o32, l32 = prep32.decode()
+        torch.cuda.synchronize()
+        sub = head0_subcase(case, (kc, vc, ks, vs) if e4m3 else None)
+        if not args.no_cpu_baseline and world == 1:
+            cpu, (ref_o, ref_l) = oracle_throughput(case, sub, args.cpu_seconds)
+        else:
+            ref_o, ref_l = oracle_head0(case, sub)
+        import numpy as np
+        eo = float(np.abs(o32[:1, :, :G].double().cpu().numpy() - ref_o).max())
+        el = float(np.abs(l32[:1, :, :G].double().cpu().numpy() - ref_l).max())
+        parity = {"max_abs_err_out_fp32": eo, "max_abs_err_lse": el,
+                  "tolerance": {"out": 2e-3, "lse": 1e-3}, "pass": eo <= 2e-3 and el <= 1e-3,
+                  "rows": f"sequence 0, KV head 0 ({G} query heads x {case.q_tokens} token(s)) "
+                          f"of the timed inputs, against the fp64 oracle"}
+
     result = None
     if rank == 0:
         peak, peak_kind = measured_peak()
@@ -362,9 +411,6 @@ def run_ours(args, rank, world, local_rank):
         achieved = nbytes / (mean_part * 1e-3) / 1e9
         value = whole_job_gbs(world, K, nbytes, total_ms)
         src_hash = kernel_source_hash()
-        cpu = None
-        if not args.no_cpu_baseline and world == 1:
-            cpu = oracle_throughput(case, args.cpu_seconds)
         e2e_gbs = world * nbytes / (statistics.fmean(t_e2e) * 1e-3) / 1e9
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
@@ -394,7 +440,12 @@ def run_ours(args, rank, world, local_rank):
                          else "fallback 6.65 TB/s",
                          "kernel": "rel_attn_partial_fp8_kernel" if e4m3 else "rel_attn_partial_kernel",
                          "traffic": load_traffic(src_hash, args.workload + ("_e4m3" if e4m3 else "")),
-                         "frac_of_8TBps_nominal": round(achieved / 8000.0, 4)},
+                         "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
+                         "frac_per_call": round(value / world / peak, 4),
+                         "frac_per_call_of_8TBps_nominal": round(value / world / 8000.0, 4),
+                         "note": "achieved/frac: the partial kernel alone; frac_per_call: the "
+                                 "whole layer-call (partial + combine) per GPU"},
+            "parity": parity,
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "us_per_call": round(statistics.fmean(t_e2e) * 1e3, 2),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

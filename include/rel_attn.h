@@ -102,8 +102,11 @@ typedef struct rel_attn_shape {
  *
  * Device-side problems (seq_len out of range, a block-table entry outside
  * the pool, a wait that exceeded its bound) do not fault: they set bits in
- * the workspace status word, read with rel_attn_read_status.  Rows of an
- * offending sequence are written as NaN.
+ * the workspace status word, read with rel_attn_read_status, and the rows
+ * they touch are written as NaN (out and lse): every row of a sequence whose
+ * seq_len is out of range; the rows of each KV head whose walk met an entry
+ * outside the pool or gave up a wait (through the combine kernel, a NaN
+ * partial makes the whole merged row NaN).
  */
 int rel_attn_decode(const rel_attn_shape* shape, const void* q,
                     const void* k_cache, const void* v_cache,
@@ -193,7 +196,8 @@ int rel_attn_partial_e4m3(const rel_attn_shape* shape, const void* q,
  *     overlap on the GPU -- on different streams, or from different host
  *     threads -- race on it; serialise them.
  *   - Device-side status is not reported (there is no workspace to read it
- *     from): rejected sequences still come back as NaN rows.
+ *     from), but the rows it concerns still come back as NaN, as described
+ *     for rel_attn_decode.
  */
 #define REL_ATTN_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
 int rel_attn_decode_static(const rel_attn_shape* shape, const void* q,
@@ -209,6 +213,15 @@ size_t rel_attn_workspace_bytes(const rel_attn_shape* shape, int num_splits);
 /* Zero the workspace status word (asynchronous on `stream`).  Call once
  * after allocating a workspace and after reading a non-zero status. */
 int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bound, in nanoseconds, of each device-side wait in launches made after
+ * this call, process-wide; 0 restores the default (2 s).  For failure-
+ * detection tests: a short bound makes waits run out, and the kernels then
+ * end with REL_ATTN_ERR_TIMEOUT in the status word and NaN rows instead of
+ * hanging.  The waits that let copies and tensor-core operations already in
+ * flight finish before a CTA exits keep a fixed 2 s bound whatever is set
+ * here.  Always returns 0. */
+int rel_attn_set_wait_limit(unsigned long long limit_ns);
 
 /* Synchronise `stream`, read the workspace status word and clear it.
  * Returns 0, REL_ATTN_ERR_TIMEOUT, REL_ATTN_ERR_BAD_SEQ or REL_ATTN_ERR_CUDA. */

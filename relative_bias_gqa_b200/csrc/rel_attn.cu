@@ -5,10 +5,13 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <numeric>
+#include <vector>
 
 #include "rel_attn.h"
 #include "rel_attn_kernels.cuh"
@@ -21,6 +24,10 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxQTokens = 8;         // query tokens per sequence (speculative verify)
 constexpr int kMaxSplits = 256;
 constexpr size_t kHeaderBytes = 256;   // status word lives here
+
+// Bound of each device-side wait of later launches (0: kDefaultTimeoutNs);
+// set by rel_attn_set_wait_limit.
+std::atomic<unsigned long long> g_wait_limit_ns{0};
 
 struct DeviceInfo {
   bool probed = false;
@@ -75,9 +82,44 @@ int validate_shape(const rel_attn_shape* s) {
   return REL_ATTN_OK;
 }
 
-// Lower edges of the tail buckets.  e_k = ceil(E * (Dmax/E)^(k/NL)) in long
-// double; a value within 1e-9 (relative) of an integer is taken as that
-// integer so that exact powers (e.g. 1024 * 2^5) do not round up.
+// Unsigned integer of arbitrary size (32-bit limbs, least significant
+// first): just enough to compare two products of powers exactly.
+struct BigUint {
+  std::vector<uint32_t> limb{1};
+  void mul(uint32_t m) {
+    uint64_t carry = 0;
+    for (auto& x : limb) {
+      const uint64_t v = (uint64_t)x * m + carry;
+      x = (uint32_t)v;
+      carry = v >> 32;
+    }
+    if (carry) limb.push_back((uint32_t)carry);
+  }
+  void mul_pow(uint32_t m, int e) { for (int i = 0; i < e; ++i) mul(m); }
+  int compare(const BigUint& o) const {
+    if (limb.size() != o.limb.size()) return limb.size() < o.limb.size() ? -1 : 1;
+    for (size_t i = limb.size(); i-- > 0;)
+      if (limb[i] != o.limb[i]) return limb[i] < o.limb[i] ? -1 : 1;
+    return 0;
+  }
+};
+
+// x >= E * (Dmax/E)^(k/n), decided exactly: with k/n = a/c in lowest terms
+// (c >= 1), the inequality is x^c >= E^(c-a) * Dmax^a between integers.
+bool at_or_above_edge(long long x, int E, int Dmax, int k, int n) {
+  if (x <= 0) return false;
+  const int g = std::gcd(k, n);
+  const int a = k / g, c = n / g;
+  BigUint lhs, rhs;
+  lhs.mul_pow((uint32_t)x, c);
+  rhs.mul_pow((uint32_t)E, c - a);
+  rhs.mul_pow((uint32_t)Dmax, a);
+  return lhs.compare(rhs) >= 0;
+}
+
+// Lower edges of the tail buckets, e_k = ceil(E * (Dmax/E)^(k/NL)), exact:
+// long double names the edge to well under one unit, and where it lies
+// within 1e-6 of an integer the integer comparison above settles it.
 // `log_scale` = NL / log2(Dmax/E): (log2(d) - log2(E)) * log_scale is the
 // tail bucket of d up to rounding, a starting guess the kernels correct
 // against the table (0 when there is a single tail bucket).
@@ -101,7 +143,14 @@ void bucket_table(const rel_attn_shape* s, int* ex, int* nl, int* edges, float* 
   for (int k = 0; k <= n; ++k) {
     const long double x = (long double)E * exp2l(lr * (long double)k / (long double)n);
     const long double r = nearbyintl(x);
-    const long double e = (fabsl(x - r) <= 1e-9L * x) ? r : ceill(x);
+    long long e;
+    if (fabsl(x - r) > 1e-6L) {
+      e = (long long)ceill(x);
+    } else {
+      e = (long long)r;
+      if (!at_or_above_edge(e, E, s->max_distance, k, n)) ++e;
+      else if (at_or_above_edge(e - 1, E, s->max_distance, k, n)) --e;
+    }
     edges[k] = (int)e;
   }
 }
@@ -358,6 +407,11 @@ int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, i
   return REL_ATTN_OK;
 }
 
+int rel_attn_set_wait_limit(unsigned long long limit_ns) {
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  return REL_ATTN_OK;
+}
+
 int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < kHeaderBytes) return REL_ATTN_ERR_INVALID_ARG;
   return cudaMemsetAsync(workspace, 0, kHeaderBytes, (cudaStream_t)stream) == cudaSuccess
@@ -430,7 +484,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->status = reinterpret_cast<unsigned*>(ws);
   prm->ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes);
   prm->ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
-  prm->timeout_ns = kDefaultTimeoutNs;
+  const unsigned long long wl = g_wait_limit_ns.load(std::memory_order_relaxed);
+  prm->timeout_ns = wl ? wl : kDefaultTimeoutNs;
   prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
   prm->num_pages = shape->num_pages;
   prm->max_pages = shape->max_pages_per_seq;

@@ -88,7 +88,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
@@ -130,6 +129,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t drain_bar = bar0 + 8u * (kB + 20);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + FC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 4);
+  volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 8);
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
@@ -153,6 +153,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *bad_page_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&p.tmap_k);
     ptx::prefetch_tmap(&p.tmap_v);
@@ -253,21 +254,19 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         ptx::mbar_arrive_expect_tx(v8full(ti % V8S), tp.npg * FC::k8PageBytes);
         ptx::tma_load_2d(st, &p.tmap_v, v8full(ti % V8S), 0, row0, pol);
         if (tp.npg > 1) ptx::tma_load_2d(st + FC::k8PageBytes, &p.tmap_v, v8full(ti % V8S), 0, row1, pol);
-        RELATTN_TRACE(0, ti);
       }
       ++nv;
     }
     if (lane == 0) {
-      if (bad_page) atomicOr(p.status, kStatusBadSeq);
-      if (!ok) {
-        // Let the copies already issued land before the CTA's memory is released.
-        volatile int never = 0;
-        for (int t = max(0, nk - K8S); t < nk; ++t)
-          ptx::mbar_wait(k8full(t % K8S), (t / K8S) & 1, &never, tlim);
-        for (int t = max(0, nv - V8S); t < nv; ++t)
-          ptx::mbar_wait(v8full(t % V8S), (t / V8S) & 1, &never, tlim);
-        if (nchunks > 0) ptx::mbar_wait(xr_full, (nchunks - 1) & 1, &never, tlim);
-      }
+      if (bad_page) *bad_page_flag = 1;
+      // Let the copies already issued land before the CTA's memory is
+      // released, on every exit (the consumers may have stopped early).
+      volatile int never = 0;
+      for (int t = max(0, nk - K8S); t < nk; ++t)
+        ptx::mbar_wait(k8full(t % K8S), (t / K8S) & 1, &never, kDrainLimitNs);
+      for (int t = max(0, nv - V8S); t < nv; ++t)
+        ptx::mbar_wait(v8full(t % V8S), (t / V8S) & 1, &never, kDrainLimitNs);
+      if (nchunks > 0) ptx::mbar_wait(xr_full, (nchunks - 1) & 1, &never, kDrainLimitNs);
     }
   }
   // ------------------------------------------------------------ converter
@@ -305,7 +304,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         return false;
       if (kc < tile_pages(ti) * kPage) widen(sbase + FC::oK8 + (ti % K8S) * FC::k8TileBytes, smem + FC::oKF, false);
       ptx::fence_proxy_async_smem();
-      if (kc == 0) RELATTN_TRACE(2, ti);
       ptx::mbar_arrive(kf_full);
       ptx::mbar_arrive(k8empty(ti % K8S));
       return true;
@@ -350,7 +348,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
         if (!ptx::mbar_wait(vf_full, j & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
-        RELATTN_TRACE(3, j);
         const uint64_t pbd = pdesc + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -386,7 +383,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
              ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
         if (!ok) break;
         ptx::tc_fence_after();
-        RELATTN_TRACE(1, i);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t ko = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
@@ -402,7 +398,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       if (ok && i > 0) ok = issue_pv(i - 1);
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
-      ptx::mbar_wait(drain_bar, 0, &never, tlim);
+      ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
     }
     __syncwarp();
   }
@@ -474,7 +470,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       const bool okw = ptx::mbar_wait(s_full + 8u * (i & 1), (i >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        RELATTN_TRACE(4, i);
         ptx::tmem_ld8(tS + lane_off + (i & 1) * N, s);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
@@ -524,7 +519,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int r = 0; r < RG; ++r) alpha_r[r] = 1.f;
       }
-      RELATTN_TRACE(5, i);
       // ---- P = exp2(x - m_ref) as f16 hi + lo parts, stacked [P_hi; P_lo],
       //      MN-major without swizzle (8-row x 16-byte core matrices)
       {
@@ -549,9 +543,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
-      RELATTN_TRACE(6, i);
       process_o(i);                            // this group's next tile is i + 2
-      RELATTN_TRACE(7, i);
       ++li;
     }
     ptx::pdl_launch_dependents();
@@ -609,8 +601,15 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   // -------------------------------------------------------------- teardown
   ptx::tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);
-  RELATTN_TRACE(17, 0);
+  // an aborted CTA, or one that met a block-table entry outside the pool,
+  // writes its rows as NaN (see the bf16 kernel)
+  const bool aborted_cta = *abort_flag != 0, bad_cta = *bad_page_flag != 0;
+  if (tid == 0) {
+    if (aborted_cta) atomicOr(p.status, kStatusTimeout);
+    if (bad_cta) atomicOr(p.status, kStatusBadSeq);
+  }
+  if (aborted_cta || bad_cta)
+    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);

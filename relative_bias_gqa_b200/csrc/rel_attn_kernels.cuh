@@ -40,19 +40,6 @@
 
 #include "sm100_ptx.cuh"
 
-// Optional timestamp hook for pipeline studies; expands to nothing unless a
-// build defines it.
-#ifndef RELATTN_TRACE
-#define RELATTN_TRACE(event, tile)
-#endif
-// Which split / KV head a block works on (the identity unless a study build
-// permutes the placement).
-#ifndef RELATTN_SPLIT_OF_BLOCK
-#define RELATTN_SPLIT_OF_BLOCK(x) (x)
-#endif
-#ifndef RELATTN_HEAD_OF_BLOCK
-#define RELATTN_HEAD_OF_BLOCK(y) (y)
-#endif
 
 namespace relattn {
 
@@ -77,6 +64,11 @@ constexpr int kPageHalfBytes = 8192;           // 64 rows x 128 B
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadSeq = 2u;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s
+// Bound of the waits that let work already issued (TMA copies, MMAs) finish
+// before a CTA releases its memory.  Fixed, whatever limit the caller sets
+// for the other waits: such work always completes, and giving up on it
+// early would free shared or tensor memory that it still writes.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;        // 2 s
 // Lazy-max slack (log2 units): p = exp2(x - m_ref) may reach 2^64, far
 // inside fp32 / bf16 range even summed over 2^31 keys.
 constexpr float kLazyLog2 = 64.f;
@@ -155,7 +147,7 @@ struct KernelConfig {
   //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[kXTables],
   //           x_empty[kXTables], drain
   static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 11 + 2 * kXTables;
-  static constexpr int oMisc = oBar + kNumBars * 8;            // tmem base, abort flag
+  static constexpr int oMisc = oBar + kNumBars * 8;            // tmem base, abort flag, bad-page flag
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAllocBytes = kBytes + 1024;            // 1024-byte alignment slack
   // TMEM columns: S[2] (N each), O[2] (2N each: the P_hi and P_lo halves),
@@ -396,7 +388,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int s_idx = RELATTN_SPLIT_OF_BLOCK(blockIdx.x), h = RELATTN_HEAD_OF_BLOCK(blockIdx.y), b = blockIdx.z;
+  const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   constexpr int NQ = T * G;
   // rows per softmax group: all NQ when the groups alternate tiles, else the
   // group's block of the column split (at most RG rows, TG tokens)
@@ -409,7 +401,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   constexpr bool kEvenSplit = KC::kAlt || T % NG == 0;
   static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(G, T) && CSp::end(kAlign) <= N &&
                                                    RG <= KC::kGR), "group width");
-  RELATTN_TRACE(16, 0);
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
@@ -451,6 +442,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * KC::kXTables);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 4);
+  volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 8);
   auto kslot = [&](int k) { return sbase + KC::oK + (uint32_t)((k % KS) * KC::kKSlotBytes); };
   auto vslot = [&](int i) { return sbase + KC::oV + (uint32_t)((i % VS) * kVSlotBytes); };
   const unsigned long long tlim = p.timeout_ns;
@@ -480,6 +472,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *bad_page_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&p.tmap_k);
     ptx::prefetch_tmap(&p.tmap_v);
@@ -588,7 +581,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
             ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
           }
-          RELATTN_TRACE(2, ti);
         }
         ++k;
       }
@@ -607,21 +599,23 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
             ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
           }
-          RELATTN_TRACE(0, tv);
         }
         i_v = tv + 1;
       }
     }
     if (lane == 0) {
-      if (bad_page) atomicOr(p.status, kStatusBadSeq);
-      if (!ok) {
-        // Let the copies already issued land before the CTA's memory is released.
-        volatile int never = 0;
-        for (int kk = max(0, k - KS); kk < k; ++kk)
-          ptx::mbar_wait(kfull(kk % KS), (kk / KS) & 1, &never, tlim);
-        for (int iv = max(0, i_v - VS); iv < i_v; ++iv)
-          ptx::mbar_wait(vfull(iv % VS), (iv / VS) & 1, &never, tlim);
-      }
+      if (bad_page) *bad_page_flag = 1;
+      // Let the copies already issued land before the CTA's memory is
+      // released.  Needed whenever the consumers may have stopped early (an
+      // expired wait anywhere in the CTA), so it is done on every exit: in a
+      // normal run these copies have landed or are about to.  Only the last
+      // KS / VS items can be in flight: issuing item k waited for item k - KS
+      // to be consumed, hence landed.
+      volatile int never = 0;
+      for (int kk = max(0, k - KS); kk < k; ++kk)
+        ptx::mbar_wait(kfull(kk % KS), (kk / KS) & 1, &never, kDrainLimitNs);
+      for (int iv = max(0, i_v - VS); iv < i_v; ++iv)
+        ptx::mbar_wait(vfull(iv % VS), (iv / VS) & 1, &never, kDrainLimitNs);
     }
   }
   // ------------------------------------------------------------ MMA issuer
@@ -644,7 +638,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
         if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
-        RELATTN_TRACE(3, j);
         const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
         const uint64_t pbd = pdesc0 + (uint64_t)(((j & 1) * KC::kPBufBytes) >> 4);
         // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
@@ -694,7 +687,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
              ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
         if (!ok) break;
         ptx::tc_fence_after();
-        RELATTN_TRACE(1, i);
         {
           const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
 #pragma unroll
@@ -713,7 +705,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       // every MMA issued so far must finish before tensor memory is released
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
-      ptx::mbar_wait(drain_bar, 0, &never, tlim);
+      ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
     }
     __syncwarp();
   }
@@ -800,7 +792,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     };
 
     int last_tile = -1;
-    RELATTN_TRACE(5, 63);
     for (int ti = 0; ti < g.ntiles; ++ti) {
       const int owner = KC::kAlt ? (ti & 1) : grp;
       const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges,
@@ -830,7 +821,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ptx::tc_fence_before();
           }
           ptx::mbar_arrive(x_empty + 8u * xb);
-          if (c == 0) RELATTN_TRACE(6, 63);
           ++c;
           if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
         }
@@ -843,7 +833,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       const bool okw = ptx::mbar_wait(s_full + 8u * (i & 1), (i >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        RELATTN_TRACE(4, i);
         ld_rows(tS + lane_off + (i & 1) * N, s);
         ptx::tc_fence_before();
       }
@@ -919,7 +908,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           else if (kl == 0 && live(r)) al_buf[r] = 1.f;
         }
       }
-      RELATTN_TRACE(5, i);
       // ---- P = exp2(x - m_ref) as bf16 hi + lo parts (~16 significant bits in
       //      the P.V product), stacked [P_hi; P_lo] = 2N rows, MN-major without
       //      swizzle: 8-row x 16-byte core matrices, row blocks 128 B apart,
@@ -971,28 +959,30 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if (KC::kAlt || grp == 0) {
         const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
         if (!any_valid) {
-          volatile int never = 0;
-          ptx::mbar_wait(vfull(i % VS), (i / VS) & 1, &never, tlim);
-          uint8_t* vrow = smem + KC::oV + (i % VS) * kVSlotBytes + kl * 128;
+          // The row is cleared after its copy has landed.  If the wait gives
+          // up (the CTA is aborting) the row is left alone: the CTA's rows
+          // are then written as NaN whatever P.V computes.
+          if (ptx::mbar_wait(vfull(i % VS), (i / VS) & 1, abort_flag, tlim)) {
+            uint8_t* vrow = smem + KC::oV + (i % VS) * kVSlotBytes + kl * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            reinterpret_cast<uint4*>(vrow)[q] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(vrow + kHalfTileBytes)[q] = make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 8; ++q) {
+              reinterpret_cast<uint4*>(vrow)[q] = make_uint4(0, 0, 0, 0);
+              reinterpret_cast<uint4*>(vrow + kHalfTileBytes)[q] = make_uint4(0, 0, 0, 0);
+            }
+          } else {
+            failed = true;
           }
         }
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
-      RELATTN_TRACE(6, i);
       if constexpr (KC::kAlt) {
         // this group's next tile is i + 2: take O(i) now
         process_o(i, alpha_r);
-        RELATTN_TRACE(7, i);
       } else {
         // every group is on every tile: take O(i-1) while P.V(i) runs
         if (last_tile >= 0) {
           process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
-          RELATTN_TRACE(7, last_tile);
         }
       }
       last_tile = i;
@@ -1085,8 +1075,18 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   // -------------------------------------------------------------- teardown
   ptx::tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort_flag) atomicOr(p.status, kStatusTimeout);
-  RELATTN_TRACE(17, 0);
+  // A CTA that gave up on a wait, or met a block-table entry outside the
+  // pool, overwrites its rows (final output, or this split's partials, which
+  // the combine kernel then propagates) with NaN: callers of the entry
+  // point without a workspace see the problem even though they cannot read
+  // the status word.
+  const bool aborted_cta = *abort_flag != 0, bad_cta = *bad_page_flag != 0;
+  if (tid == 0) {
+    if (aborted_cta) atomicOr(p.status, kStatusTimeout);
+    if (bad_cta) atomicOr(p.status, kStatusBadSeq);
+  }
+  if (aborted_cta || bad_cta)
+    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, KC::kTmemCols);

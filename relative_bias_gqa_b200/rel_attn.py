@@ -28,6 +28,7 @@ EXPORTED = (
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
     "rel_attn_split_pages", "rel_attn_decode_e4m3", "rel_attn_partial_e4m3",
+    "rel_attn_set_wait_limit",
 )
 
 
@@ -78,6 +79,8 @@ def _load():
     lib.rel_attn_split_pages.argtypes = [SP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.rel_attn_split_pages.restype = ctypes.c_int
+    lib.rel_attn_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    lib.rel_attn_set_wait_limit.restype = ctypes.c_int
     lib.rel_attn_error_string.argtypes = [ctypes.c_int]
     lib.rel_attn_error_string.restype = ctypes.c_char_p
     lib.rel_attn_version.argtypes = []
@@ -140,6 +143,11 @@ def rel_attn_split_pages(shape: RelAttnShape, seq_len: int, window: int, num_spl
     if rc != REL_ATTN_OK:
         raise RelAttnError(rc)
     return a.value, b.value
+
+
+def rel_attn_set_wait_limit(limit_ns: int) -> None:
+    """Bound of each device-side wait in later launches (0: the 2 s default)."""
+    lib.rel_attn_set_wait_limit(int(limit_ns))
 
 
 def _stream_ptr(stream) -> int:

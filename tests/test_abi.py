@@ -69,6 +69,33 @@ def test_host_bucket_every_distance_nb1280(ra):
     assert np.array_equal(got, oracle.bucket_of_distance(d, 1280))
 
 
+# (NB, E, Dmax) triples: the standard tables, the geometries the GPU parity
+# tests run, dense tables where consecutive edges repeat, and extremes of the
+# integer ranges.  Exact powers (E * (Dmax/E)^(k/NL) an integer) must not
+# round up: 1024 * 2^(10k/256) is an integer at k = 0, 128, 256.
+EDGE_TRIPLES = [
+    (1280, 1024, 1 << 20), (1030, 1024, 1 << 20), (1536, 1024, 1 << 20),
+    (364, 64, 5000), (200, 16, 100000), (600, 100, 1500), (1024 + 512, 1024, (1 << 31) - 1),
+    (513, 1, (1 << 31) - 1), (1100, 1000, 1000 * 3 ** 4), (1088, 1024, 1 << 30),
+]
+
+
+@pytest.mark.parametrize("nb,e,dmax", EDGE_TRIPLES, ids=[str(t) for t in EDGE_TRIPLES])
+def test_host_edges_exact_for_other_geometries(ra, nb, e, dmax):
+    """The library's edge table (long double, settled by exact integer
+    comparison near integers) equals the oracle's exact-integer edges: each
+    edge, and the distances one either side, get the same bucket."""
+    import oracle
+    s = shape(ra, num_buckets=nb, exact_buckets=e, max_distance=dmax)
+    edges = oracle.log_bucket_edges(nb, e, dmax)
+    d = np.unique(np.concatenate([edges - 1, edges, edges + 1, np.arange(0, min(e + 10, 4000)),
+                                  [dmax - 1, dmax, dmax + 1]]))
+    d = d[(d >= 0) & (d < (1 << 31) - 1)]
+    want = oracle.bucket_of_distance(d, nb, e, dmax)
+    got = np.array([ra.rel_attn_bucket(s, int(x)) for x in d])
+    assert np.array_equal(got, want)
+
+
 BAD = [
     dict(q_tokens=0), dict(q_tokens=9), dict(head_dim=64), dict(page_size=16),
     dict(num_q_heads=47), dict(num_q_heads=24), dict(num_q_heads=40), dict(num_q_heads=56),

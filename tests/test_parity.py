@@ -221,11 +221,19 @@ def test_sliding_100k(ra):
             check(*run_gpu(ra, case, splits), *ref)
 
 
-def test_full_100k_with_split_sweep(ra):
+def test_full_100k_every_split_count(ra):
+    """The 100K full-attention decode with every split count 1..256 (and the
+    heuristic's) against one oracle result."""
     case = W.make_workload("full_100k", seed=0, device="cuda")
     ref = run_oracle(case)
-    for s in list(range(1, 65)) + [72, 96, 128, 148, 200, 255, 256, 0]:
-        check(*run_gpu(ra, case, s), *ref)
+    shape = ra.shape_of(case.q, case.k_cache, case.block_table, case.rel_table, out_fp32=True)
+    from relative_bias_gqa_b200.rel_attn import Workspace
+    ws = Workspace.for_shape(shape, 256, "cuda")
+    worst = (0.0, 0.0)
+    for s in list(range(1, 257)) + [0]:
+        eo, el = check(*run_gpu(ra, case, s, workspace=ws), *ref)
+        worst = (max(worst[0], eo), max(worst[1], el))
+    assert ws.read_status() == ra.REL_ATTN_OK
 
 
 def test_verify_t8_256k(ra):
@@ -256,14 +264,110 @@ def _sub_case(case, idx):
         seq_lens=case.seq_lens[idx].cpu(), rel_table=case.rel_table.cpu())
 
 
-def test_batched_32_sampled(ra):
+def test_batched_32_every_sequence(ra):
+    """All 32 sequences of the mixed-length batch against the oracle, one
+    sequence at a time on the host (a compact copy of its pages keeps the
+    fp64 working set small)."""
     case = W.make_workload("batched_32", seed=0, device="cuda")
-    idx = [0, 5, 17, 31]
-    sub = _sub_case(case, idx)
-    ref_o, ref_l = run_oracle(sub)
-    for splits in (1, 3, 0):
+    runs = [run_gpu(ra, case, splits) for splits in (1, 3, 0)]
+    for b in range(case.batch):
+        ref_o, ref_l = run_oracle(_sub_case(case, [b]))
+        for out, lse in runs:
+            check(out[b:b + 1], lse[b:b + 1], ref_o, ref_l)
+
+
+# ------------------------------------------- full-size key sets and poison
+def _zero_q_r_bits_v(case):
+    """Q = 0 and R = 0 (uniform weights over the selected keys) and V row of
+    position j holding the bits of j in its first 18 dims (0/1, exact in
+    bf16), on every KV head, through the case's shuffled block table."""
+    case.q.zero_()
+    case.rel_table.zero_()
+    P = case.page_size
+    for b in range(case.batch):
+        L = int(case.seq_lens[b])
+        pos = torch.arange(L, device="cuda")
+        bits = ((pos[:, None] >> torch.arange(18, device="cuda")[None]) & 1).to(torch.bfloat16)
+        pages = case.block_table[b].long()[pos // P]
+        vals = torch.zeros(L, 128, dtype=torch.bfloat16, device="cuda")
+        vals[:, :18] = bits
+        for h in range(case.num_kv_heads):
+            case.v_cache[pages, h, pos % P] = vals
+
+
+def _check_key_sets(case, out, lse, one_split):
+    """Each row must select exactly its key set J (a contiguous position
+    range).  One split: exp(lse) = |J| (to the nearest integer up to 16,384
+    keys, else to 4e-6 relative: fp32 log2 / exp rounding) and out[c] =
+    #{j in J : bit c of j} / |J| to a quarter of 1/|J| -- the partial
+    kernel's sums of 0/1 values are exact and out is one rounded division,
+    so a key missing, added or swapped moves some out[c] by about 1/(2|J|).
+    Several splits: the merge's fp32 weights carry ~1e-6 relative error, so
+    the check resolves whole pages (64 keys: >= 1e-5 relative at 262,144
+    keys), which is what a split boundary can get wrong."""
+    T, W = case.q_tokens, case.window
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    for b in range(case.batch):
+        L = int(case.seq_lens[b])
+        for t in range(T):
+            p = L - T + t
+            lo = 0 if W <= 0 else max(0, p - W + 1)
+            n = p - lo + 1
+            cnt = np.array([_bit_count_range(lo, p, c) for c in range(18)], dtype=np.float64)
+            est = np.exp(l[b, t])
+            strict = one_split or n <= 16384      # merge error ~1e-6 << 1/(4|J|)
+            if strict and n <= 16384:
+                assert np.all(np.round(est) == n), (b, t, est, n)
+            else:
+                rel = 4e-6 if strict else 1e-5
+                assert np.all(np.abs(est / n - 1.0) <= rel), (b, t, est, n)
+            err = np.abs(o[b, t, :, :18] - cnt[None] / n).max()
+            tol = 0.25 / n if strict else max(0.25 / n, 4e-6)
+            assert err <= tol, (b, t, err, tol)
+
+
+def _bit_count_range(lo, hi, c):
+    """#{j in [lo, hi] : bit c of j is set}, in closed form."""
+    def upto(x):                                   # over [0, x)
+        period = 1 << (c + 1)
+        return (x // period) * (1 << c) + max(0, x % period - (1 << c))
+    return upto(hi + 1) - upto(lo)
+
+
+@pytest.mark.parametrize("name", ["full_100k", "sliding_100k", "verify_t8_256k"])
+def test_key_set_identity_full_size(ra, name):
+    case = W.make_workload(name, seed=2, device="cuda")
+    _zero_q_r_bits_v(case)
+    for splits in (1, 5, 0):
         out, lse = run_gpu(ra, case, splits)
-        check(out[idx], lse[idx], ref_o, ref_l)
+        _check_key_sets(case, out, lse, one_split=splits == 1)
+
+
+@pytest.mark.parametrize("name", ["full_100k", "sliding_100k", "verify_t8_256k"])
+def test_poisoned_slots_full_size(ra, name):
+    """NaN in every pool page no sequence owns (64 of them, shuffled in among
+    the owned ones), in the slots past L and before the window: the outputs
+    are bit-identical to the clean run and match the oracle."""
+    case = W.make_workload(name, seed=3, device="cuda", extra_pages=64)
+    ref = run_oracle(case)
+    bad = W.poison_unused(case)
+    for splits in (1, 7, 0):
+        clean = run_gpu(ra, case, splits)
+        dirty = run_gpu(ra, bad, splits)
+        assert torch.equal(clean[0], dirty[0]) and torch.equal(clean[1], dirty[1])
+        check(*dirty, *ref)
+
+
+@pytest.mark.parametrize("T", [2, 3, 4, 5, 6, 7])
+def test_verify_256k_every_token_count(ra, T):
+    """Full-size speculative verify for every token count below 8 (G = 6; one
+    KV head keeps the oracle fast, the sequence still spans every split)."""
+    case = W.make_case(seq_lens=[262_144], q_tokens=T, num_q_heads=6, num_kv_heads=1,
+                       window=0, num_buckets=1280, seed=T).to("cuda")
+    ref = run_oracle(case)
+    for splits in (1, 18, 0):
+        check(*run_gpu(ra, case, splits), *ref)
 
 
 # ------------------------------------------------------------- error paths
@@ -278,6 +382,68 @@ def test_bad_sequence_length_reports_and_writes_nan(ra):
         assert torch.isnan(out).all() and torch.isnan(lse).all()
         assert ws.read_status() == ra.REL_ATTN_ERR_BAD_SEQ
         assert ws.read_status() == ra.REL_ATTN_OK    # reading clears it
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_block_table_entry_outside_pool_writes_nan(ra, splits):
+    """One block-table entry of sequence 0 points outside the pool: every row
+    of sequence 0 comes back NaN (all its KV heads walk that page) and the
+    status says BAD_SEQ; sequence 1 is untouched and still matches the
+    oracle.  Both through the workspace entry and the allocation-free one."""
+    import ctypes
+    from relative_bias_gqa_b200.rel_attn import Workspace
+    case = small(0, T=2, Hkv=2, lens=[2000, 1500])
+    ref_o, ref_l = run_oracle(case, batch_indices=[1])
+    for bad_entry in (case.k_cache.shape[0] + 7, -3):
+        case.block_table[0, 5] = bad_entry
+        shape = ra.shape_of(case.q, case.k_cache, case.block_table, case.rel_table,
+                            max_seq_len=case.max_seq_len, out_fp32=True)
+        ws = Workspace.for_shape(shape, splits, "cuda")
+        out, lse = run_gpu(ra, case, splits, workspace=ws)
+        assert torch.isnan(out[0]).all() and torch.isnan(lse[0]).all()
+        check(out[1:], lse[1:], ref_o[1:], ref_l[1:])
+        assert ws.read_status() == ra.REL_ATTN_ERR_BAD_SEQ
+        out2 = torch.zeros_like(out)
+        lse2 = torch.zeros_like(lse)
+        rc = ra.lib.rel_attn_decode_static(
+            ctypes.byref(shape), case.q.data_ptr(), case.k_cache.data_ptr(),
+            case.v_cache.data_ptr(), case.block_table.data_ptr(), case.seq_lens.data_ptr(),
+            case.rel_table.data_ptr(), case.window, splits, out2.data_ptr(), lse2.data_ptr(),
+            torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        assert rc == ra.REL_ATTN_OK
+        assert torch.isnan(out2[0]).all() and torch.isnan(lse2[0]).all()
+        assert torch.equal(out2[1:], out[1:]) and torch.equal(lse2[1:], lse[1:])
+
+
+@pytest.mark.parametrize("workload,T", [("full_100k", 1), ("verify_t8_256k", 8)])
+def test_injected_wait_limit_times_out_cleanly(ra, workload, T):
+    """A 1 us bound on every device wait makes the waits for TMA copies run
+    out: the call must come back promptly with REL_ATTN_ERR_TIMEOUT in the
+    status word and NaN rows (never a hang), and the next call with the
+    default bound must be correct again on the same workspace."""
+    import time
+    from relative_bias_gqa_b200.rel_attn import Workspace
+    case = W.make_workload(workload, seed=4, device="cuda", num_q_heads=6 * 2, num_kv_heads=2)
+    assert case.q_tokens == T
+    shape = ra.shape_of(case.q, case.k_cache, case.block_table, case.rel_table,
+                        max_seq_len=case.max_seq_len, out_fp32=True)
+    ws = Workspace.for_shape(shape, 0, "cuda")
+    run_gpu(ra, case, 0, workspace=ws)                   # warm: attributes, tensor maps
+    assert ws.read_status() == ra.REL_ATTN_OK
+    try:
+        ra.rel_attn_set_wait_limit(1000)
+        t0 = time.perf_counter()
+        out, lse = run_gpu(ra, case, 0, workspace=ws)
+        elapsed = time.perf_counter() - t0
+    finally:
+        ra.rel_attn_set_wait_limit(0)
+    assert elapsed < 1.0, elapsed                        # far below the 2 s default bound
+    assert ws.read_status() == ra.REL_ATTN_ERR_TIMEOUT
+    assert torch.isnan(out).any() and torch.isnan(lse).any()
+    assert ws.read_status() == ra.REL_ATTN_OK            # reading cleared it
+    check(*run_gpu(ra, case, 0, workspace=ws), *run_oracle(case))
+    assert ws.read_status() == ra.REL_ATTN_OK
 
 
 def test_status_clean_after_normal_call(ra):

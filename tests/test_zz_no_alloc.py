@@ -53,9 +53,13 @@ def _reference_call(ra, case, num_splits):
 
 
 def test_static_entry_matches_workspace_entry_two_calls_in_a_row(ra):
+    """Both entry points launch the same kernels with the same split count,
+    so their results must be bit-identical; the first case also runs more
+    splits than the second, so the second call finds the first one's
+    partials still in the shared array."""
     cases = [
         (W.make_case(seq_lens=[5000], q_tokens=1, num_q_heads=48, num_kv_heads=8,
-                     window=0, num_buckets=1280, seed=3).to("cuda"), 7),
+                     window=0, num_buckets=1280, seed=3).to("cuda"), 37),
         (W.make_case(seq_lens=[2500, 900], q_tokens=3, num_q_heads=12, num_kv_heads=2,
                      window=1024, num_buckets=1024, seed=4).to("cuda"), 0),
     ]
@@ -65,10 +69,27 @@ def test_static_entry_matches_workspace_entry_two_calls_in_a_row(ra):
         torch.cuda.synchronize()
         ref_out, ref_lse = _reference_call(ra, case, splits)
         torch.cuda.synchronize()
-        eo = (out - ref_out).abs().max().item()
-        el = (lse - ref_lse).abs().max().item()
-        assert np.isfinite(eo) and eo <= OUT_TOL, eo
-        assert np.isfinite(el) and el <= LSE_TOL, el
+        assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+
+
+def test_static_entry_against_the_oracle(ra):
+    """The allocation-free call checked directly against the fp64 oracle, with
+    one split (no partials: the kernel writes the output itself), then with
+    several splits after a call that used more of the array."""
+    import oracle
+    case = W.make_case(seq_lens=[3001, 64, 129], q_tokens=2, num_q_heads=18, num_kv_heads=3,
+                       window=0, num_buckets=1280, seed=6).to("cuda")
+    ref_o, ref_l = oracle.rel_attn_decode_ref(case.q, case.k_cache, case.v_cache,
+                                              case.block_table, case.seq_lens,
+                                              case.rel_table, case.window)
+    for splits in (1, 40, 5, 1):
+        rc, out, lse = _static_call(ra, case, splits)
+        assert rc == ra.REL_ATTN_OK, ra.error_string(rc)
+        torch.cuda.synchronize()
+        eo = np.abs(out.double().cpu().numpy() - ref_o).max()
+        el = np.abs(lse.double().cpu().numpy() - ref_l).max()
+        assert np.isfinite(eo) and eo <= OUT_TOL, (splits, eo)
+        assert np.isfinite(el) and el <= LSE_TOL, (splits, el)
 
 
 def test_static_entry_rejects_shapes_beyond_its_scratch(ra):
