@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for relative-bias GQA decode attention.
+"""fp64 CPU oracle for relative-bias GQA decode attention and the KV-cache
+producer step that feeds it.
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
 ``bench.py`` (its ``cpu_baseline`` leg and its ``--impl reference`` arm) may
@@ -22,4 +23,11 @@ from .rel_attn_ref import (  # noqa: F401
     e4m3_to_float,
     dequant_kv,
     rel_attn_decode_fp8kv_ref,
+)
+from .kv_write_ref import (  # noqa: F401
+    short_conv_ref,
+    short_conv_fp32,
+    bf16_rne,
+    e4m3_rne_satfinite,
+    kv_write_ref,
 )
