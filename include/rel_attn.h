@@ -62,10 +62,11 @@ extern "C" {
 /* Problem shape.  All fields are host integers. */
 typedef struct rel_attn_shape {
   int batch;             /* B >= 1                                              */
-  int q_tokens;          /* T, query tokens per sequence, 1..8 (verify steps)  */
+  int q_tokens;          /* T, query tokens per sequence, 1..9 (verify steps)  */
   int num_q_heads;       /* Hq                                                  */
   int num_kv_heads;      /* Hkv, Hq % Hkv == 0, G = Hq/Hkv in {4, 6, 8};
-                            T <= 8 for G = 4 and 6, T <= 6 for G = 8          */
+                            T <= 9 for G = 4 and 6, T <= 8 for G = 8 (at most
+                            64 query rows G*T per KV head)                     */
   int head_dim;          /* D, must be 128                                      */
   int page_size;         /* P, must be 64                                       */
   int num_pages;         /* pages in the K/V pool                               */
@@ -205,6 +206,55 @@ int rel_attn_decode_static(const rel_attn_shape* shape, const void* q,
                            const int32_t* block_table, const int32_t* seq_lens,
                            const void* rel_table, int window, int num_splits,
                            void* out, float* lse, void* stream);
+
+/*
+ * rel_attn_kv_write -- the producer step that fills the cache the decode
+ * reads: a short convolution over the new tokens' K and V, written into the
+ * paged KV cache (bf16, or E4M3 codes), with the raw K/V kept for the next
+ * steps' convolutions.  One kernel.
+ *
+ * "vLLM TML Inkling 지원", section "TML Inkling 모델 아키텍처": every layer
+ * applies a short convolution of window 4 to the attention keys and to the
+ * attention values; section "Sconv 캐시 및 TP 샤딩": the convolution state
+ * is kept by the unified KV-cache manager as the cache of a virtual
+ * sliding-window layer, channel by channel.  The pages give no formula;
+ * this library reads it as a causal depthwise convolution over positions:
+ *   k~[p][h][c] = sum_{i=0..3} w[0][h][c][i] * k[p-i][h][c]   (k[q < 0] = 0)
+ * and likewise for V with w[1].  The sum is formed in fp32 with the taps in
+ * the order i = 0, 1, 2, 3, then rounded to nearest even (bf16), or divided
+ * by the KV head's scale and rounded to nearest even E4M3 (saturating at
+ * +-448).
+ *
+ * shape       reads batch, q_tokens (T = new tokens per sequence, 1..2^24),
+ *             num_kv_heads, head_dim (128), page_size (64), num_pages and
+ *             max_pages_per_seq; the other fields are ignored.
+ *   k_new     bf16 [B, T, Hkv, D]: the new tokens' keys before the
+ *   v_new     convolution (positions L_b - T .. L_b - 1), and values.
+ *   conv_w    bf16 [2, Hkv, D, 4]: the K taps, then the V taps; tap i
+ *             multiplies the vector at position p - i.
+ *   k_raw     bf16 [num_pages, Hkv, P, D]: the sconv cache, the raw K and V
+ *   v_raw     of every position, addressed by block_table like the KV
+ *             cache.  Positions before L_b - T are read (the last three);
+ *             the new positions are written.
+ *   k_cache   [num_pages, Hkv, P, D]: the KV cache the decode reads; bf16,
+ *   v_cache   or uint8 E4M3 codes when k_scale / v_scale are given.
+ *   k_scale   fp32 [Hkv] per-KV-head scales (both, or both NULL for bf16).
+ *   v_scale
+ *   block_table, seq_lens   as for rel_attn_decode: seq_lens[b] = L_b
+ *             counts the T new tokens (T <= L_b <= max_pages_per_seq * P).
+ *   workspace NULL, or a workspace as for rel_attn_decode (256-byte
+ *             aligned, initialised): a sequence whose length or block-table
+ *             entries are out of range sets REL_ATTN_ERR_BAD_SEQ in its
+ *             status word.  The new tokens of such a sequence that touch a
+ *             bad entry are not written.
+ * All device pointers are caller-owned, 16-byte aligned (4 for the int32
+ * and fp32 arrays).  Asynchronous on `stream`; nothing is allocated.
+ */
+int rel_attn_kv_write(const rel_attn_shape* shape, const void* k_new, const void* v_new,
+                      const void* conv_w, void* k_raw, void* v_raw, void* k_cache,
+                      void* v_cache, const float* k_scale, const float* v_scale,
+                      const int32_t* block_table, const int32_t* seq_lens,
+                      void* workspace, void* stream);
 
 /* Bytes of workspace rel_attn_decode needs for this shape and split count
  * (num_splits <= 0: the heuristic's choice).  0 when the shape is invalid. */

@@ -16,12 +16,12 @@
 #include "rel_attn.h"
 #include "rel_attn_kernels.cuh"
 #include "rel_attn_fp8.cuh"
+#include "rel_attn_kvwrite.cuh"
 
 namespace relattn {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxQTokens = 8;         // query tokens per sequence (speculative verify)
 constexpr int kMaxSplits = 256;
 constexpr size_t kHeaderBytes = 256;   // status word lives here
 
@@ -307,7 +307,7 @@ int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t 
     return REL_ATTN_ERR_INVALID_ARG;                  // no instance for this shape
   } else {
     constexpr int NG = softmax_groups(G, T);
-    using KC = KernelConfig<N, NG, G>;
+    using KC = KernelConfig<N, NG, G, T>;
     auto kern = rel_attn_partial_kernel<N, G, NG, T>;
     constexpr int smem = KC::kAllocBytes;
     bool& attr = di.attr_set[G / 2 - 2][T - 1];
@@ -334,6 +334,7 @@ int launch_partial_group(const DecodeParams& prm, int T, int S, int B, int Hkv, 
     case 6: return launch_partial<G, 6>(prm, S, B, Hkv, st, di);
     case 7: return launch_partial<G, 7>(prm, S, B, Hkv, st, di);
     case 8: return launch_partial<G, 8>(prm, S, B, Hkv, st, di);
+    case 9: return launch_partial<G, 9>(prm, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }
@@ -634,6 +635,65 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, flo
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The KV-cache producer step: short convolution over the new tokens' K and V,
+// paged KV-cache write, optional E4M3 quantisation (rel_attn_kvwrite.cuh).
+// ---------------------------------------------------------------------------
+extern "C" int rel_attn_kv_write(const rel_attn_shape* shape, const void* k_new, const void* v_new,
+                                 const void* conv_w, void* k_raw, void* v_raw, void* k_cache,
+                                 void* v_cache, const float* k_scale, const float* v_scale,
+                                 const int32_t* block_table, const int32_t* seq_lens,
+                                 void* workspace, void* stream) {
+  const rel_attn_shape* s = shape;
+  if (!s) return REL_ATTN_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->batch > 65535 || s->q_tokens < 1 || s->q_tokens > (1 << 24) ||
+      s->num_kv_heads < 1 || s->num_kv_heads > 65535 || s->head_dim != kHeadDim ||
+      s->page_size != kPage || s->num_pages < 1 || s->max_pages_per_seq < 1)
+    return REL_ATTN_ERR_INVALID_ARG;
+  if ((long long)s->num_pages * s->num_kv_heads * kPage >= (1ll << 31) ||
+      (long long)s->max_pages_per_seq * kPage >= (1ll << 31))
+    return REL_ATTN_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !conv_w || !k_raw || !v_raw || !k_cache || !v_cache || !block_table ||
+      !seq_lens)
+    return REL_ATTN_ERR_INVALID_ARG;
+  const bool e4m3 = k_scale != nullptr;
+  if (e4m3 != (v_scale != nullptr)) return REL_ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+  if (misaligned(k_new, 16) || misaligned(v_new, 16) || misaligned(conv_w, 16) ||
+      misaligned(k_raw, 16) || misaligned(v_raw, 16) || misaligned(k_cache, 16) ||
+      misaligned(v_cache, 16) || misaligned(block_table, 4) || misaligned(seq_lens, 4) ||
+      (e4m3 && (misaligned(k_scale, 4) || misaligned(v_scale, 4))) ||
+      (workspace && misaligned(workspace, 256)))
+    return REL_ATTN_ERR_INVALID_ARG;
+  int dev;
+  int rc = probe_device(&dev);
+  if (rc != REL_ATTN_OK) return rc;
+  KvWriteParams prm;
+  prm.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+  prm.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  prm.conv_w = reinterpret_cast<const __nv_bfloat16*>(conv_w);
+  prm.k_raw = reinterpret_cast<__nv_bfloat16*>(k_raw);
+  prm.v_raw = reinterpret_cast<__nv_bfloat16*>(v_raw);
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.k_scale = k_scale;
+  prm.v_scale = v_scale;
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.status = reinterpret_cast<unsigned*>(workspace);
+  prm.B = s->batch;
+  prm.T = s->q_tokens;
+  prm.Hkv = s->num_kv_heads;
+  prm.num_pages = s->num_pages;
+  prm.max_pages = s->max_pages_per_seq;
+  const dim3 grid((unsigned)((s->q_tokens + kKvwTokensPerCta - 1) / kKvwTokensPerCta),
+                  (unsigned)s->num_kv_heads, (unsigned)s->batch);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (e4m3) rel_attn_kv_write_kernel<true><<<grid, kKvwThreads, 0, st>>>(prm);
+  else rel_attn_kv_write_kernel<false><<<grid, kKvwThreads, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------------------
 // Allocation-free entry point.

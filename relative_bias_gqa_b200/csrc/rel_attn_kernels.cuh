@@ -45,6 +45,7 @@ namespace relattn {
 
 constexpr int kHeadDim = 128;
 constexpr int kPage = 64;
+constexpr int kMaxQTokens = 9;                 // query tokens per sequence (speculative verify)
 constexpr int kTileKeys = 128;                 // two pages per tile
 constexpr int kMaxTailBuckets = 512;           // log buckets supported
 constexpr int kSoftmaxThreads = 128;           // one softmax group
@@ -54,9 +55,10 @@ constexpr int kBarSetup = 6;                   // every warp but the producer (p
 // Softmax groups of the instance for G heads per KV head and T query tokens:
 // four from six tokens on where each group then carries at most 12 rows of
 // S^T (a thread's per-tile work halves and every SM sub-partition runs four
-// softmax warps to hide each other's latencies), else two.
+// softmax warps to hide each other's latencies), and always past 48 query
+// rows (the 64-wide instances); else two.
 __host__ __device__ constexpr int softmax_groups(int G, int T) {
-  return (T >= 6 && (T + 3) / 4 * G <= 12) ? 4 : 2;
+  return (T >= 6 && ((T + 3) / 4 * G <= 12 || G * T > 48)) ? 4 : 2;
 }
 constexpr int kVSlotBytes = 32768;             // V tile: 128 keys x 128 dims bf16
 constexpr int kHalfTileBytes = 16384;          // 128 rows x 128 B (one 64-dim half)
@@ -104,20 +106,22 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 
 // Compile-time configuration of one kernel instance: N = padded group width
 // (G heads x T tokens rounded up to the MMA N step), NG = softmax groups,
-// G = query heads per KV head.
+// G = query heads per KV head, T = query tokens.
 // K tiles and relative-row chunks share one ring of slots (each slot is
 // released as soon as its MMA has read it); V tiles have their own, deeper
 // ring (a V slot is held until the P.V product of its tile).
-template <int N, int NG, int G>
+template <int N, int NG, int G, int T>
 struct KernelConfig {
   // N = 16 (one token): the softmax groups alternate tiles, each with all the
-  // rows.  N = 32 / 48 (2..8 tokens): every group takes every tile, each with
-  // its own block of rows (a column split of S^T, X^T and O^T).
+  // rows.  N = 32 / 48 / 64 (2..9 tokens): every group takes every tile, each
+  // with its own block of rows (a column split of S^T, X^T and O^T).
   static constexpr bool kAlt = (N == 16);
   static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
   static constexpr int kConsumers = kAlt ? kSoftmaxThreads : kSoftmaxThreads * NG;  // arrivals per tile
   static constexpr int kXTables = kAlt ? NG : 1;               // relative chunks in flight (X, Y)
-  static constexpr int kGR = kAlt ? N : N / NG;                // row capacity of a group
+  // row capacity of a group: N / NG, or more when the tokens do not split
+  // evenly (nine tokens over four groups: one group takes three)
+  static constexpr int kGR = kAlt ? N : ((T + NG - 1) / NG * G > N / NG ? (T + NG - 1) / NG * G : N / NG);
   // relative rows per chunk: 128 cover one 128-key tile for one token; with
   // T tokens a tile needs 127 + T rows
   static constexpr int kRows = (N == 16) ? 128 : 136;
@@ -127,6 +131,10 @@ struct KernelConfig {
   // P.V), so the one-token instance gives V four of its six 32 KB slots.
   static constexpr int kKSlots = 2;
   static constexpr int kVSlots = (N == 16) ? 4 : (N == 32 ? 3 : 2);
+  // P buffers: two, so that the softmax writes P(i+1) while P.V(i) still
+  // reads P(i); the 64-wide instances keep one to fit shared memory (their
+  // softmax then takes O(i-1), which proves P.V(i-1) done, before writing P(i))
+  static constexpr int kPBufs = (N == 64) ? 1 : 2;
   static constexpr int kVLag = 0;                               // V issued this many tiles after K
   // Relative-table gather stride: odd for conflict-free gathers.  The N = 16
   // instance serves G live rows (one token).
@@ -137,8 +145,8 @@ struct KernelConfig {
   static constexpr int oK = 0;
   static constexpr int oV = kKSlots * kKSlotBytes;
   static constexpr int oQ = oV + kVSlots * kVSlotBytes;
-  static constexpr int oP = oQ + kOperandBytes;                // two P buffers
-  static constexpr int oY = oP + 2 * kPBufBytes;               // one table per relative chunk in flight
+  static constexpr int oP = oQ + kOperandBytes;                // kPBufs P buffers
+  static constexpr int oY = oP + kPBufs * kPBufBytes;          // one table per relative chunk in flight
   static constexpr int oRed = oY + kXTables * kYBytes;         // [NG][2][4][kGR]
   static constexpr int oAlpha = oRed + NG * 2 * 4 * kGR * 4;   // [NG][2][kGR]
   static constexpr int oEdges = oAlpha + NG * 2 * kGR * 4;
@@ -158,7 +166,9 @@ struct KernelConfig {
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
   static_assert(kKSlotBytes >= 2 * kHalfTileBytes && oV % 1024 == 0 && oQ % 1024 == 0,
                 "slot layout");
-  static_assert(oV >= NG * kGR * 128 * 4 * 2 + NG * kGR * 4 * 2, "epilogue exchange area");
+  // the epilogue exchanges the groups' rows through the K and V rings (idle
+  // by then)
+  static_assert(oQ >= NG * kGR * 128 * 4 * 2 + NG * kGR * 4 * 2, "epilogue exchange area");
 };
 
 // Column split of the query rows among NG softmax groups (T >= 2): group q
@@ -191,16 +201,19 @@ struct ColSplit {
 
 // Group width N of the instance for G heads per KV head and T tokens (0: not
 // supported): 16 for one token (the alternating-group instance, G <= 8);
-// otherwise the smaller of 32 and 48 whose query slots hold every softmax
-// group's row block 8-aligned, else the smaller one that holds them 4-aligned.
+// otherwise the smallest of 32, 48 and 64 whose query slots hold every softmax
+// group's row block 8-aligned, else the smallest that holds them 4-aligned
+// (64 only past 48 rows: G = 8 with 7 or 8 tokens, G = 6 with 9).
 __host__ __device__ constexpr int group_width_for(int G, int T) {
-  if (G < 1 || G > 8 || T < 1 || T > 8) return 0;
+  if (G < 1 || G > 8 || T < 1 || T > kMaxQTokens) return 0;
   if (T == 1) return 16;
   const int NG = softmax_groups(G, T);
   if (cs_end(T, G, NG, 8) <= 32) return 32;
   if (cs_end(T, G, NG, 8) <= 48) return 48;
   if (cs_end(T, G, NG, 4) <= 32) return 32;
   if (cs_end(T, G, NG, 4) <= 48) return 48;
+  if (G * T > 48 && cs_end(T, G, NG, 8) <= 64) return 64;
+  if (G * T > 48 && cs_end(T, G, NG, 4) <= 64) return 64;
   return 0;
 }
 
@@ -373,9 +386,9 @@ __device__ void fill_rows(const DecodeParams& p, int b, int h, int s, float o_va
 // T (query tokens) is a template parameter: every per-row loop below runs
 // over the NQ = T*G live rows only, fully unrolled.
 template <int N, int G, int NG, int T>
-__global__ void __launch_bounds__(KernelConfig<N, NG, G>::kThreads, 1)
+__global__ void __launch_bounds__(KernelConfig<N, NG, G, T>::kThreads, 1)
 rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
-  using KC = KernelConfig<N, NG, G>;
+  using KC = KernelConfig<N, NG, G, T>;
   constexpr int KS = KC::kKSlots;
   constexpr int VS = KC::kVSlots;
   constexpr int ROWS = KC::kRows;
@@ -639,7 +652,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
         const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
-        const uint64_t pbd = pdesc0 + (uint64_t)(((j & 1) * KC::kPBufBytes) >> 4);
+        const uint64_t pbd = pdesc0 + (uint64_t)(((j % KC::kPBufs) * KC::kPBufBytes) >> 4);
         // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -916,11 +929,16 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       //      group's units end before the next group's slots).  Rows past the
       //      group's live ones get zeros; slots no group owns are never read
       //      back, as O^T column n depends on P row n only.
+      if constexpr (KC::kPBufs == 1) {
+        // one P buffer: P.V(i-1) must have read it before P(i) goes in, and
+        // taking O(i-1) waits for exactly that
+        if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
+      }
       {
         constexpr int U = kAlign;                              // rows per store
         constexpr int NU = (RG + U - 1) / U;
         const int nu = kEvenSplit ? NU : (nrows + U - 1) / U;
-        const uint32_t pbuf = sP0 + (uint32_t)((i & 1) * KC::kPBufBytes);
+        const uint32_t pbuf = sP0 + (uint32_t)((i % KC::kPBufs) * KC::kPBufBytes);
         const uint32_t pkey = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16);
 #pragma unroll
         for (int cb = 0; cb < NU; ++cb) {
@@ -979,7 +997,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if constexpr (KC::kAlt) {
         // this group's next tile is i + 2: take O(i) now
         process_o(i, alpha_r);
-      } else {
+      } else if constexpr (KC::kPBufs == 2) {
         // every group is on every tile: take O(i-1) while P.V(i) runs
         if (last_tile >= 0) {
           process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);

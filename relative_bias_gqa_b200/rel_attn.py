@@ -28,7 +28,7 @@ EXPORTED = (
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
     "rel_attn_split_pages", "rel_attn_decode_e4m3", "rel_attn_partial_e4m3",
-    "rel_attn_set_wait_limit",
+    "rel_attn_set_wait_limit", "rel_attn_kv_write",
 )
 
 
@@ -79,6 +79,8 @@ def _load():
     lib.rel_attn_split_pages.argtypes = [SP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.rel_attn_split_pages.restype = ctypes.c_int
+    lib.rel_attn_kv_write.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, P, P]
+    lib.rel_attn_kv_write.restype = ctypes.c_int
     lib.rel_attn_set_wait_limit.argtypes = [ctypes.c_ulonglong]
     lib.rel_attn_set_wait_limit.restype = ctypes.c_int
     lib.rel_attn_error_string.argtypes = [ctypes.c_int]
@@ -189,7 +191,7 @@ def rel_attn_decode(q, k_cache, v_cache, block_table, seq_lens, rel_table,
     q bf16 [B, T, Hq, D]; k_cache / v_cache bf16 [num_pages, Hkv, P, D];
     block_table int32 [B, max_pages]; seq_lens int32 [B]; rel_table bf16
     [Hkv, NB, D] -- all contiguous CUDA tensors.  Returns (out, lse).
-    Supported: D = 128, P = 64, Hq / Hkv in {4, 6, 8} with T <= 8 (T <= 6
+    Supported: D = 128, P = 64, Hq / Hkv in {4, 6, 8} with T <= 9 (T <= 8
     for 8); other shapes raise RelAttnError (REL_ATTN_ERR_INVALID_ARG).
     """
     for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
@@ -253,6 +255,44 @@ def rel_attn_decode_e4m3(q, k_codes, v_codes, k_scale, v_scale, block_table, seq
     if rc != REL_ATTN_OK:
         raise RelAttnError(rc)
     return out, lse
+
+
+def rel_attn_kv_write(k_new, v_new, conv_w, k_raw, v_raw, k_cache, v_cache, block_table,
+                      seq_lens, k_scale=None, v_scale=None, workspace: Optional[Workspace] = None,
+                      stream=None):
+    """The KV-cache producer step (see include/rel_attn.h): short convolution
+    of the T new tokens' K/V (k_new / v_new bf16 [B, T, Hkv, D], taps conv_w
+    bf16 [2, Hkv, D, 4]), raw K/V into the sconv cache k_raw / v_raw, the
+    convolved K/V into k_cache / v_cache (bf16, or uint8 / float8_e4m3fn
+    E4M3 codes with k_scale / v_scale fp32 [Hkv]).  In place; returns None."""
+    if k_cache.dtype == torch.float8_e4m3fn:
+        k_cache = k_cache.view(torch.uint8)
+    if v_cache.dtype == torch.float8_e4m3fn:
+        v_cache = v_cache.view(torch.uint8)
+    e4m3 = k_scale is not None
+    cache_dt = torch.uint8 if e4m3 else torch.bfloat16
+    checks = [("k_new", k_new, torch.bfloat16), ("v_new", v_new, torch.bfloat16),
+              ("conv_w", conv_w, torch.bfloat16), ("k_raw", k_raw, torch.bfloat16),
+              ("v_raw", v_raw, torch.bfloat16), ("k_cache", k_cache, cache_dt),
+              ("v_cache", v_cache, cache_dt), ("block_table", block_table, torch.int32),
+              ("seq_lens", seq_lens, torch.int32)]
+    if e4m3:
+        checks += [("k_scale", k_scale, torch.float32), ("v_scale", v_scale, torch.float32)]
+    for name, t, dt in checks:
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    B, T, Hkv, D = k_new.shape
+    shape = make_shape(batch=B, q_tokens=T, num_q_heads=Hkv, num_kv_heads=Hkv,
+                       num_pages=k_cache.shape[0], max_pages_per_seq=block_table.shape[1],
+                       num_buckets=1, head_dim=D, page_size=k_cache.shape[2])
+    rc = lib.rel_attn_kv_write(
+        ctypes.byref(shape), k_new.data_ptr(), v_new.data_ptr(), conv_w.data_ptr(),
+        k_raw.data_ptr(), v_raw.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        k_scale.data_ptr() if e4m3 else None, v_scale.data_ptr() if e4m3 else None,
+        block_table.data_ptr(), seq_lens.data_ptr(),
+        workspace.buf.data_ptr() if workspace is not None else None, _stream_ptr(stream))
+    if rc != REL_ATTN_OK:
+        raise RelAttnError(rc)
 
 
 class Prepared:

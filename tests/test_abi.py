@@ -97,9 +97,9 @@ def test_host_edges_exact_for_other_geometries(ra, nb, e, dmax):
 
 
 BAD = [
-    dict(q_tokens=0), dict(q_tokens=9), dict(head_dim=64), dict(page_size=16),
+    dict(q_tokens=0), dict(q_tokens=10), dict(head_dim=64), dict(page_size=16),
     dict(num_q_heads=47), dict(num_q_heads=24), dict(num_q_heads=40), dict(num_q_heads=56),
-    dict(num_q_heads=80), dict(num_q_heads=64, q_tokens=7), dict(num_q_heads=64, q_tokens=8),
+    dict(num_q_heads=80), dict(num_q_heads=64, q_tokens=9),
     dict(num_kv_heads=0), dict(batch=0),
     dict(num_buckets=0), dict(num_buckets=1024 + 513), dict(num_pages=0),
     dict(max_pages_per_seq=0), dict(out_fp32=2), dict(max_seq_len=-1),
@@ -118,11 +118,11 @@ def test_invalid_shape_rejected_before_any_cuda_call(ra, kw):
 
 
 # Group sizes with instances: 48/8 (G = 6), the previous Inkling's 64/8 full
-# (G = 8, up to 6 tokens: 8 x 6 rows fill the 48 query slots) and 64/16
-# sliding (G = 4) layers.
-GOOD = [dict(num_q_heads=48, num_kv_heads=8, q_tokens=t) for t in range(1, 9)] + \
-       [dict(num_q_heads=64, num_kv_heads=8, q_tokens=t) for t in range(1, 7)] + \
-       [dict(num_q_heads=64, num_kv_heads=16, q_tokens=t) for t in range(1, 9)]
+# (G = 8, up to 8 tokens: 8 x 8 rows fill the 64 query slots) and 64/16
+# sliding (G = 4) layers; nine tokens for G = 4 and 6.
+GOOD = [dict(num_q_heads=48, num_kv_heads=8, q_tokens=t) for t in range(1, 10)] + \
+       [dict(num_q_heads=64, num_kv_heads=8, q_tokens=t) for t in range(1, 9)] + \
+       [dict(num_q_heads=64, num_kv_heads=16, q_tokens=t) for t in range(1, 10)]
 
 
 @pytest.mark.parametrize("kw", GOOD, ids=[f"{k['num_q_heads']}/{k['num_kv_heads']}-T{k['q_tokens']}" for k in GOOD])

@@ -18,7 +18,7 @@ PROGRAM = r"""
 using namespace relattn;
 int main() {
   for (int G = 1; G <= 8; ++G) {
-    for (int T = 1; T <= 8; ++T) {
+    for (int T = 1; T <= 9; ++T) {
       const int N = group_width_for(G, T), NG = softmax_groups(G, T);
       const int A = (T == 1) ? 8 : (cs_end(T, G, NG, 8) <= N ? 8 : 4);
       std::printf("%d %d %d %d %d", G, T, N, NG, A);
@@ -52,20 +52,29 @@ def table(tmp_path_factory):
     return rows
 
 
-SUPPORTED = [(6, t) for t in range(1, 9)] + [(8, t) for t in range(1, 7)] + [(4, t) for t in range(1, 9)]
+SUPPORTED = [(6, t) for t in range(1, 10)] + [(8, t) for t in range(1, 9)] + [(4, t) for t in range(1, 10)]
 
 
 def test_supported_shapes_have_instances(table):
     for G, T in SUPPORTED:
-        assert table[(G, T)][0] in (16, 32, 48), (G, T)
-    assert table[(8, 7)][0] == 0 and table[(8, 8)][0] == 0       # 56 / 64 rows > 48 slots
+        assert table[(G, T)][0] in (16, 32, 48, 64), (G, T)
+    assert table[(8, 9)][0] == 0                                  # 72 rows > 64 slots
 
 
 def test_inkling2_instances(table):
-    # 48/8 heads: N and group counts of the measured instances
-    assert [table[(6, t)][0] for t in range(1, 9)] == [16, 32, 32, 32, 48, 48, 48, 48]
-    assert [table[(6, t)][1] for t in range(1, 9)] == [2, 2, 2, 2, 2, 4, 4, 4]
-    assert [table[(6, t)][2] for t in range(6, 9)] == [8, 4, 4]       # 4-aligned at T = 7, 8
+    # 48/8 heads: N and group counts of the measured instances; nine tokens
+    # (an 8-head MTP chain's verify step) need the 64-wide instance
+    assert [table[(6, t)][0] for t in range(1, 10)] == [16, 32, 32, 32, 48, 48, 48, 48, 64]
+    assert [table[(6, t)][1] for t in range(1, 10)] == [2, 2, 2, 2, 2, 4, 4, 4, 4]
+    assert [table[(6, t)][2] for t in range(6, 10)] == [8, 4, 4, 4]    # 4-aligned at T = 7..9
+
+
+def test_wide_instances(table):
+    # 64/8 heads with 7 and 8 tokens: four groups of up to 16 rows, 8-aligned
+    assert [table[(8, t)][:3] for t in (7, 8)] == [(64, 4, 8), (64, 4, 8)]
+    # nine tokens over four groups: 2/2/2/3 tokens, the last group 18 rows
+    assert [g[2] for g in table[(6, 9)][3]] == [12, 12, 12, 18]
+    assert table[(4, 9)][:2] == (48, 4)
 
 
 @pytest.mark.parametrize("G,T", [k for k in SUPPORTED if k[1] >= 2])
@@ -82,8 +91,9 @@ def test_column_split_layout(table, G, T):
         end = slot + -(-rows // A) * A
         nxt = groups[q + 1][1] if q + 1 < NG else N
         assert end <= nxt <= N
-        # at most the per-group row capacity of the instance
-        assert rows <= N // NG
+        # at most the per-group row capacity of the instance (N / NG, or
+        # ceil(T / NG) * G when the tokens do not split evenly)
+        assert rows <= max(N // NG, -(-T // NG) * G)
         # tensor-memory loads: RG = the instance's row capacity per group,
         # read as 8-column loads from the slot (A = 8) or from the 8-aligned
         # column below it, RG + 4 columns (A = 4); they must end inside the

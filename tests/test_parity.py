@@ -126,7 +126,7 @@ def test_split_count_invariance_small(ra):
 
 # --------------------------------------------------- exact key-set identity
 @pytest.mark.parametrize("T,window,L", [(1, 0, 1000), (3, 77, 1000), (8, 0, 333), (8, 1024, 3000),
-                                         (1, 1024, 2500), (2, 5, 129)])
+                                         (1, 1024, 2500), (2, 5, 129), (9, 0, 700), (9, 100, 2000)])
 def test_key_set_identity_bit_exact(ra, T, window, L):
     """Q = 0 and R = 0 give uniform weights: exp(lse) is the number of keys a
     row selects and out * |J| counts, per bit c < 18, the selected positions
@@ -155,7 +155,7 @@ def test_key_set_identity_bit_exact(ra, T, window, L):
 
 def test_poisoned_slots_do_not_matter(ra):
     for kw in (dict(L=3001, T=1, window=0), dict(L=2500, T=8, window=1024, NB=1024),
-               dict(L=1500, T=3, window=100)):
+               dict(L=1500, T=3, window=100), dict(L=2222, T=9, window=0)):
         case = small(**kw)
         ref = run_oracle(case)
         for splits in (1, 4):
@@ -466,8 +466,12 @@ def small_g(L, G, T=1, window=0, NB=1280, seed=0, Hkv=2, lens=None, **kw):
 
 
 GROUP_CASES = (
-    [dict(G=8, T=t, L=L) for t in range(1, 7) for L in (t, 129, 2100)] +
-    [dict(G=4, T=t, L=L) for t in range(1, 9) for L in (t, 129, 2100)] +
+    [dict(G=8, T=t, L=L) for t in range(1, 9) for L in (t, 129, 2100)] +
+    [dict(G=4, T=t, L=L) for t in range(1, 10) for L in (t, 129, 2100)] +
+    [dict(G=6, T=9, L=L) for L in (9, 10, 129, 2100, 5000)] +
+    [dict(G=8, T=8, L=3000, window=1024, NB=1024), dict(G=8, T=7, L=2500, window=100),
+     dict(G=6, T=9, L=3000, window=1024, NB=1024), dict(G=4, T=9, L=1700, window=512, NB=1024),
+     dict(G=6, T=9, L=3000, NB=200, exact_buckets=16, max_distance=100000)] +
     [dict(G=8, T=1, L=3001, window=1024, NB=1024), dict(G=8, T=6, L=3000, window=100),
      dict(G=4, T=1, L=3001, window=512, NB=1024), dict(G=4, T=8, L=2500, window=512, NB=1024),
      dict(G=4, T=5, L=1500, window=64), dict(G=8, T=3, L=5000, seed=3),
@@ -484,7 +488,7 @@ def test_other_group_sizes(ra, kw):
         check(*run_gpu(ra, case, splits), *ref)
 
 
-@pytest.mark.parametrize("G,T", [(8, 2), (8, 6), (4, 3), (4, 8)])
+@pytest.mark.parametrize("G,T", [(8, 2), (8, 6), (8, 8), (4, 3), (4, 8), (6, 9), (4, 9)])
 def test_other_group_sizes_batched(ra, G, T):
     case = small_g(0, G, T=T, Hkv=3, lens=[T, 64, 65 + T, 300, 1111, 2049, 129, T + 1])
     ref = run_oracle(case)
@@ -500,7 +504,7 @@ def test_previous_model_layers_100k(ra, name):
         check(*run_gpu(ra, case, splits), *ref)
 
 
-@pytest.mark.parametrize("G,T", [(8, 6), (4, 8)])
+@pytest.mark.parametrize("G,T", [(8, 6), (4, 8), (8, 7), (8, 8), (6, 9), (4, 9)])
 def test_other_group_sizes_verify_256k(ra, G, T):
     """Full-size verify with the G = 8 / G = 4 instances (one KV head keeps the
     oracle fast; the sequence still spans every split)."""
