@@ -153,11 +153,12 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
  *                     head h is e4m3(k_code) * k_scale[h], likewise for V.
  * Every other argument, the workspace and the outputs are as for
  * rel_attn_decode / rel_attn_partial (rel_attn_combine merges the splits of
- * either).  The kernels widen the codes to f16 on chip (exact) and run the
- * query through f16 for q.k (exact for |q| in [2^-14, 65504]; smaller
- * magnitudes round to f16 subnormals); the relative term stays bf16.
- * Current limits: shape->q_tokens must be 1 and Hq/Hkv must be 6 (else
- * REL_ATTN_ERR_INVALID_ARG).
+ * either).  The E4M3 tiles go to the tensor cores as they are (E4M3 x E4M3
+ * MMAs, fp32 accumulation): the query is carried as two E4M3 terms scaled
+ * per row by a power of two (exact for a bf16 query), the softmax weights
+ * as three (12 significant bits); the relative term stays bf16.
+ * Current limits: shape->q_tokens must be 1 and Hq/Hkv must be 4, 6 or 8
+ * (else REL_ATTN_ERR_INVALID_ARG).
  */
 int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q,
                          const void* k_cache, const void* v_cache,

@@ -34,7 +34,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   bool attr_set[3][kMaxQTokens] = {};     // [G = 4, 6, 8][T - 1]
-  bool attr_fp8 = false;
+  bool attr_fp8[3] = {};                   // [G = 4, 6, 8]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -445,7 +445,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
   if (kv_e4m3) {
-    if (shape->q_tokens != 1 || shape->num_q_heads != 6 * shape->num_kv_heads || !k_scale || !v_scale ||
+    if (shape->q_tokens != 1 || !k_scale || !v_scale ||
         (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))
       return REL_ATTN_ERR_INVALID_ARG;
   }
@@ -513,17 +513,31 @@ int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int
   }
 }
 
-int launch_partial_e4m3(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
-  using FC = Fp8Config;
-  auto kern = rel_attn_partial_fp8_kernel<6>;
-  if (!di.attr_fp8) {
+// (templates cannot have C linkage; this block sits inside extern "C")
+extern "C++" template <int G>
+int launch_partial_e4m3_g(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
+  using FC = Fp8Config<G>;
+  auto kern = rel_attn_partial_fp8_kernel<G>;
+  bool& attr = di.attr_fp8[G / 2 - 2];
+  if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kAllocBytes) != cudaSuccess)
       return REL_ATTN_ERR_CUDA;
-    di.attr_fp8 = true;
+    attr = true;
   }
   dim3 grid(S, Hkv, B);
   kern<<<grid, FC::kThreads, FC::kAllocBytes, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
+}
+
+int launch_partial_e4m3(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
+                        DeviceInfo& di) {
+  const int B = shape->batch, Hkv = shape->num_kv_heads;
+  switch (shape->num_q_heads / Hkv) {
+    case 4: return launch_partial_e4m3_g<4>(prm, S, B, Hkv, st, di);
+    case 6: return launch_partial_e4m3_g<6>(prm, S, B, Hkv, st, di);
+    case 8: return launch_partial_e4m3_g<8>(prm, S, B, Hkv, st, di);
+    default: return REL_ATTN_ERR_INVALID_ARG;
+  }
 }
 
 // LSE-merge launch; programmatic dependent launch lets it start while the
@@ -597,7 +611,7 @@ int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q, const void*
                    out, lse, workspace, workspace_bytes, &prm, &S, &di, k_scale, v_scale, true);
   if (rc != REL_ATTN_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  rc = launch_partial_e4m3(prm, S, shape->batch, shape->num_kv_heads, st, *di);
+  rc = launch_partial_e4m3(prm, shape, S, st, *di);
   if (rc != REL_ATTN_OK || S == 1) return rc;
   return launch_combine(shape, S, out, lse, workspace, st);
 }
@@ -614,8 +628,7 @@ int rel_attn_partial_e4m3(const rel_attn_shape* shape, const void* q, const void
   int rc = prepare(shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, num_splits,
                    out, lse, workspace, workspace_bytes, &prm, &S, &di, k_scale, v_scale, true);
   if (rc != REL_ATTN_OK) return rc;
-  return launch_partial_e4m3(prm, S, shape->batch, shape->num_kv_heads,
-                             reinterpret_cast<cudaStream_t>(stream), *di);
+  return launch_partial_e4m3(prm, shape, S, reinterpret_cast<cudaStream_t>(stream), *di);
 }
 
 int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, float* lse,

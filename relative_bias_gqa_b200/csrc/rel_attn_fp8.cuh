@@ -6,79 +6,88 @@
 // the bytes of the bandwidth-bound decode.  Codes are OFP8 E4M3, one fp32
 // scale per KV head for K and one for V (k = e4m3(code) * k_scale[h]).
 //
-// Tensor-core MMAs take both operands in the same 16-bit type, and the
-// query must not lose precision, so the tiles are widened on chip:
-//   warp 0        TMA producer: E4M3 K and V page tiles (8 KB per page) into
-//                 two staging rings, relative-row chunks into their own slot.
-//   warp 1        MMA issuer: S^T = K16 . Qh^T and O^T = V16^T . [P_hi; P_lo]^T
-//                 in f16 (E4M3 -> f16 is exact; Qh is the query in f16),
-//                 X^T = R_chunk . Q^T in bf16 as in the bf16 kernel.
-//   warps 2..9    two softmax groups alternating tiles (as the one-token bf16
-//                 kernel), P in f16 hi + lo parts.
-//   warps 10..13  converter: one thread per key row widens the staged E4M3 K
-//                 and V rows to f16 (cvt.rn.f16x2.e4m3x2, exact) into the
-//                 MMA's 128B-swizzled layouts, zeroing V rows no query may see.
-// The K scale multiplies the S logits, the V scale the final output.  The
-// softmax's lazy reference max lets P grow to 2^14 here (f16 range).
+// The E4M3 page tiles are the tensor-core operands themselves
+// (tcgen05.mma kind::f8f6f4, both operands E4M3): nothing is widened on
+// chip.  Neither the query nor P may lose precision, so each is carried as
+// a short sum of E4M3 terms, each term scaled into E4M3 range and given its
+// own rows of the MMA's N side:
+//   S^T = K8 . [Q_hi; Q_lo]^T       q * 2^e_r = Q_hi + Q_lo / 16, exact for a
+//                                   bf16 query (8 significant bits = 4 + 4)
+//   O^T = V8^T . [P_hi; P_mid; P_lo]^T   P = P_hi + P_mid / 16 + P_lo / 256,
+//                                   12 significant bits
+//   X^T = R_chunk . Q^T             bf16 (kind::f16) as in the bf16 kernel
+// Roles as in the bf16 one-token kernel: warp 0 TMA producer (K8 and V8
+// page tiles, 8 KB per page, and relative-row chunks, each in its own
+// ring), warp 1 MMA issuer, two softmax groups of 4 warps alternating tiles.
+// The K scale and the query's per-row power of two fold into the logit
+// scale, the V scale into the output.  The lazy reference max keeps
+// P <= 2^8 here, inside E4M3 range.
 #pragma once
 
 namespace relattn {
 
+template <int G>
 struct Fp8Config {
-  static constexpr int N = 16, NG = 2, NQ = 6, RG = 6, ROWS = 128;
-  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + 128;
-  static constexpr int kK8Slots = 3, kV8Slots = 3;
-  static constexpr int k8TileBytes = 128 * 128;                 // 128 keys x 128 B
-  static constexpr int k8PageBytes = 64 * 128;
-  static constexpr int kF16TileBytes = 2 * kHalfTileBytes;      // 128 keys x 256 B
-  static constexpr int kRHalfBytes = ROWS * 128;
-  static constexpr int kYStride = 7;
+  static constexpr int N = 16;                                  // S^T / X^T columns
+  static constexpr int NP = 32;                                 // P.V columns: 3 terms x G rows
+  static constexpr int NG = 2, RG = G;
+  static_assert(2 * G <= N && 3 * G <= NP && G % 2 == 0, "group size");
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
+  static constexpr int kKSlots = 3, kVSlots = 5, kRSlots = 2;
+  static constexpr int kTile8 = 128 * 128;                      // 128 keys x 128 B
+  static constexpr int kPage8 = 64 * 128;
+  static constexpr int kRHalf = 128 * 128;                      // 128 rows x 64 dims bf16
+  static constexpr int kRBytes = 2 * kRHalf;
+  static constexpr int kYStride = G + 1;
   static constexpr int kGR = 8;
-  static constexpr int kPBufBytes = 2 * (2 * N * 128);          // [P_hi; P_lo]: 128 keys x 2N rows f16
-  static constexpr int kYBytes = align_up(ROWS * kYStride * 4, 16);
-  static constexpr int oK8 = 0;
-  static constexpr int oV8 = oK8 + kK8Slots * k8TileBytes;
-  static constexpr int oXR = oV8 + kV8Slots * k8TileBytes;      // relative-row chunk (bf16)
-  static constexpr int oKF = oXR + 2 * kRHalfBytes;             // K tile widened to f16
-  static constexpr int oVF = oKF + kF16TileBytes;               // V tile widened to f16
-  static constexpr int oQ = oVF + kF16TileBytes;                // Q bf16 (for X)
-  static constexpr int oQh = oQ + 2 * N * 128;                  // Q f16 (for S)
-  static constexpr int oP = oQh + 2 * N * 128;                  // two P buffers
+  static constexpr int kPBufBytes = 128 * NP;                   // 128 keys x 32 B
+  static constexpr int kYBytes = align_up(128 * kYStride * 4, 16);
+  static constexpr int oK = 0;
+  static constexpr int oV = oK + kKSlots * kTile8;
+  static constexpr int oR = oV + kVSlots * kTile8;
+  static constexpr int oQ8 = oR + kRSlots * kRBytes;            // [Q_hi; Q_lo; 0]: 16 rows x 128 B
+  static constexpr int oQ = oQ8 + N * 128;                      // bf16 Q for X: 16 rows x 256 B
+  static constexpr int oP = oQ + 2 * N * 128;                   // two P buffers
   static constexpr int oY = oP + 2 * kPBufBytes;                // one table per group
   static constexpr int oRed = oY + NG * kYBytes;                // [NG][2][4][kGR]
-  static constexpr int oAlpha = oRed + NG * 2 * 4 * kGR * 4;    // [NG][2][kGR] (unused slack)
-  static constexpr int oEdges = oAlpha + NG * 2 * kGR * 4;
+  static constexpr int oQf = oRed + NG * 2 * 4 * kGR * 4;       // per-row logit factors [G]
+  static constexpr int oEdges = oQf + 64;
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
-  // k8full[3] k8empty[3] v8full[3] v8empty[3] kf_full kf_empty vf_full vf_empty
-  // xr_full xr_empty s_full[2] s_empty[2] p_full[2] o_full[2] o_empty[2]
-  // x_full[2] x_empty[2] drain
-  static constexpr int kNumBars = 2 * kK8Slots + 2 * kV8Slots + 6 + 14 + 1;
-  static constexpr int oMisc = oBar + kNumBars * 8;
+  // kfull/kempty[KS] vfull/vempty[VS] rfull/rempty[RS] s_full/s_empty[2]
+  // p_full[2] o_full/o_empty[2] x_full/x_empty[2] drain
+  static constexpr int kNumBars = 2 * (kKSlots + kVSlots + kRSlots) + 4 + 2 + 4 + 4 + 1;
+  static constexpr int oMisc = oBar + kNumBars * 8;             // tmem base, abort, bad page
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAllocBytes = kBytes + 1024;
   static constexpr int kTmemCols = 128;                         // S[2] 32 + O[2] 64 + X[2] 32
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
-  static_assert(oKF % 1024 == 0 && oVF % 1024 == 0 && oXR % 1024 == 0 && oQ % 1024 == 0 &&
-                oQh % 1024 == 0 && oV8 % 1024 == 0, "slot alignment");
-  static_assert(oXR >= NG * RG * 128 * 4 * 2 + NG * RG * 4 * 2, "epilogue exchange area");
+  static_assert(oV % 1024 == 0 && oR % 1024 == 0 && oQ8 % 1024 == 0 && oQ % 1024 == 0,
+                "operand alignment");
+  static_assert(oV >= NG * RG * 128 * 4 * 2 + NG * RG * 4 * 2, "epilogue exchange area");
 };
 
-// E4M3 pair (low 16 bits) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)v));
+// E4M3 codes of (lo, hi), round to nearest even, saturating; lo in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// The two values of an E4M3 pair (low byte first), exactly.
+__device__ __forceinline__ float2 e4m3x2_value(uint32_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)v));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 template <int G>
-__global__ void __launch_bounds__(Fp8Config::kThreads, 1)
+__global__ void __launch_bounds__(Fp8Config<G>::kThreads, 1)
 rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
-  using FC = Fp8Config;
-  constexpr int N = FC::N, NG = FC::NG, NQ = FC::NQ, RG = FC::RG, ROWS = FC::ROWS;
+  using FC = Fp8Config<G>;
+  constexpr int N = FC::N, NP = FC::NP, NG = FC::NG, RG = FC::RG;
   constexpr int YS = FC::kYStride;
-  constexpr int K8S = FC::kK8Slots, V8S = FC::kV8Slots;
+  constexpr int KS = FC::kKSlots, VS = FC::kVSlots, RS = FC::kRSlots;
   constexpr int T = 1;
-  static_assert(NQ == G * T, "one token, six heads");
+  constexpr float kLazy8 = 8.f;               // P = exp2(x - m_ref) <= 2^8 < 448
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -110,38 +119,36 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 
   // --------------------------------------------------------- smem carve-up
   int* s_edges = reinterpret_cast<int*>(smem + FC::oEdges);
+  float* qf = reinterpret_cast<float*>(smem + FC::oQf);
   const uint32_t bar0 = sbase + FC::oBar;
-  auto k8full = [&](int s) { return bar0 + 8u * s; };
-  auto k8empty = [&](int s) { return bar0 + 8u * (K8S + s); };
-  auto v8full = [&](int s) { return bar0 + 8u * (2 * K8S + s); };
-  auto v8empty = [&](int s) { return bar0 + 8u * (2 * K8S + V8S + s); };
-  constexpr int kB = 2 * K8S + 2 * V8S;
-  const uint32_t kf_full = bar0 + 8u * (kB + 0), kf_empty = bar0 + 8u * (kB + 1);
-  const uint32_t vf_full = bar0 + 8u * (kB + 2), vf_empty = bar0 + 8u * (kB + 3);
-  const uint32_t xr_full = bar0 + 8u * (kB + 4), xr_empty = bar0 + 8u * (kB + 5);
-  const uint32_t s_full = bar0 + 8u * (kB + 6);     // +8*buf
-  const uint32_t s_empty = bar0 + 8u * (kB + 8);
-  const uint32_t p_full = bar0 + 8u * (kB + 10);
-  const uint32_t o_full = bar0 + 8u * (kB + 12);
-  const uint32_t o_empty = bar0 + 8u * (kB + 14);
-  const uint32_t x_full = bar0 + 8u * (kB + 16);    // +8*group
-  const uint32_t x_empty = bar0 + 8u * (kB + 18);
-  const uint32_t drain_bar = bar0 + 8u * (kB + 20);
+  auto kfull = [&](int s) { return bar0 + 8u * s; };
+  auto kempty = [&](int s) { return bar0 + 8u * (KS + s); };
+  auto vfull = [&](int s) { return bar0 + 8u * (2 * KS + s); };
+  auto vempty = [&](int s) { return bar0 + 8u * (2 * KS + VS + s); };
+  auto rfull = [&](int s) { return bar0 + 8u * (2 * KS + 2 * VS + s); };
+  auto rempty = [&](int s) { return bar0 + 8u * (2 * KS + 2 * VS + RS + s); };
+  constexpr int kB = 2 * (KS + VS + RS);
+  const uint32_t s_full = bar0 + 8u * (kB + 0);     // +8*buf
+  const uint32_t s_empty = bar0 + 8u * (kB + 2);
+  const uint32_t p_full = bar0 + 8u * (kB + 4);
+  const uint32_t o_full = bar0 + 8u * (kB + 6);
+  const uint32_t o_empty = bar0 + 8u * (kB + 8);
+  const uint32_t x_full = bar0 + 8u * (kB + 10);    // +8*group
+  const uint32_t x_empty = bar0 + 8u * (kB + 12);
+  const uint32_t drain_bar = bar0 + 8u * (kB + 14);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + FC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 4);
   volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 8);
+  auto kslot = [&](int i) { return sbase + FC::oK + (uint32_t)((i % KS) * FC::kTile8); };
+  auto vslot = [&](int i) { return sbase + FC::oV + (uint32_t)((i % VS) * FC::kTile8); };
+  auto rslot = [&](int c) { return sbase + FC::oR + (uint32_t)((c % RS) * FC::kRBytes); };
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
   if (tid == 0) {
-    for (int s = 0; s < K8S; ++s) { ptx::mbar_init(k8full(s), 1); ptx::mbar_init(k8empty(s), 128); }
-    for (int s = 0; s < V8S; ++s) { ptx::mbar_init(v8full(s), 1); ptx::mbar_init(v8empty(s), 128); }
-    ptx::mbar_init(kf_full, 128);
-    ptx::mbar_init(kf_empty, 1);
-    ptx::mbar_init(vf_full, 128);
-    ptx::mbar_init(vf_empty, 1);
-    ptx::mbar_init(xr_full, 1);
-    ptx::mbar_init(xr_empty, 1);
+    for (int s = 0; s < KS; ++s) { ptx::mbar_init(kfull(s), 1); ptx::mbar_init(kempty(s), 1); }
+    for (int s = 0; s < VS; ++s) { ptx::mbar_init(vfull(s), 1); ptx::mbar_init(vempty(s), 1); }
+    for (int s = 0; s < RS; ++s) { ptx::mbar_init(rfull(s), 1); ptx::mbar_init(rempty(s), 1); }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(s_full + 8u * i, 1);
       ptx::mbar_init(s_empty + 8u * i, kSoftmaxThreads);
@@ -165,37 +172,68 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     if (warp == 1) {
       ptx::tmem_alloc(ptx::smem_addr(tmem_holder), FC::kTmemCols);
       ptx::tmem_relinquish();
-    } else if (warp < 10) {
-      // Q group tile, twice (bf16 for the relative product, f16 for S):
-      // rows n = g (padding rows zero), 128B-swizzled K-major.
-      const int st = tid - 64;
+    } else {
+      const int st = tid - 64;                  // softmax thread 0..255
+      const int sw = st >> 5;                   // its warp 0..7
+      // bf16 Q for X: rows 0..G-1 the group's heads, other rows zero,
+      // 128B-swizzled K-major in two 64-dim halves
       for (int u = st; u < N * 16; u += kSoftmaxThreads * NG) {
         const int n = u >> 4, half = (u >> 3) & 1, w16 = u & 7;
-        uint4 v = make_uint4(0, 0, 0, 0), vh = make_uint4(0, 0, 0, 0);
-        if (n < NQ) {
-          const __nv_bfloat16* src = p.q + ((size_t)b * p.Hq + h * G + n) * kHeadDim + half * 64 + w16 * 8;
-          v = __ldg(reinterpret_cast<const uint4*>(src));
-          const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-          __half2* h2 = reinterpret_cast<__half2*>(&vh);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) h2[e] = __float22half2_rn(__bfloat1622float2(q2[e]));
-        }
-        const int off = half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4);
-        *reinterpret_cast<uint4*>(smem + FC::oQ + off) = v;
-        *reinterpret_cast<uint4*>(smem + FC::oQh + off) = vh;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < G)
+          v = __ldg(reinterpret_cast<const uint4*>(
+              p.q + ((size_t)b * p.Hq + h * G + n) * kHeadDim + half * 64 + w16 * 8));
+        *reinterpret_cast<uint4*>(smem + FC::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4)) = v;
       }
+      // E4M3 Q: warp w < G splits head row w.  q * 2^e (e puts the row's
+      // largest |q| in [128, 256)) = Q_hi + Q_lo / 16: Q_hi the nearest E4M3
+      // value, Q_lo the E4M3 code of 16 x the remainder (at most four
+      // significant bits of a bf16 query remain, so the sum is exact down to
+      // 2^-10 x the row maximum).  Rows G..2G-1 hold Q_lo, the rest zero.
+      if (sw < G) {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+            p.q + ((size_t)b * p.Hq + h * G + sw) * kHeadDim + lane * 4));
+        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        const float2 a = __bfloat1622float2(q2[0]), c = __bfloat1622float2(q2[1]);
+        float mx = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(c.x), fabsf(c.y)));
+        mx = warp_max(mx);
+        int e = 0;
+        if (mx > 0.f) {
+          int ex;
+          frexpf(mx, &ex);                      // mx = m 2^ex, m in [0.5, 1)
+          e = 8 - ex;                           // mx 2^e in [128, 256)
+        }
+        const float sc = ldexpf(1.f, e);
+        const float x0 = a.x * sc, x1 = a.y * sc, x2 = c.x * sc, x3 = c.y * sc;
+        const uint32_t h01 = e4m3x2_rn(x0, x1), h23 = e4m3x2_rn(x2, x3);
+        const float2 v01 = e4m3x2_value(h01), v23 = e4m3x2_value(h23);
+        const uint32_t l01 = e4m3x2_rn((x0 - v01.x) * 16.f, (x1 - v01.y) * 16.f);
+        const uint32_t l23 = e4m3x2_rn((x2 - v23.x) * 16.f, (x3 - v23.y) * 16.f);
+        const int chunk = lane >> 2, sub = (lane & 3) * 4;
+        auto put = [&](int n, uint32_t w) {
+          *reinterpret_cast<uint32_t*>(smem + FC::oQ8 + n * 128 + ((chunk ^ (n & 7)) << 4) + sub) = w;
+        };
+        put(sw, h01 | (h23 << 16));
+        put(G + sw, l01 | (l23 << 16));
+        // logit factor of this row: the K scale, the 2^-e of the split and
+        // log2(e) / sqrt(D)
+        if (lane == 0) qf[sw] = __ldg(p.k_scale + h) * ldexpf(1.f, -e) * p.scale_log2;
+      } else {
+        // rows 2G..15 are zero
+        for (int u = (sw - G) * 32 + lane; u < (N - 2 * G) * 32; u += (8 - G) * 32)
+          *reinterpret_cast<uint32_t*>(smem + FC::oQ8 + (2 * G + u / 32) * 128 + (u % 32) * 4) = 0u;
+      }
+      for (int e = st; e <= p.nl; e += kSoftmaxThreads * NG) s_edges[e] = p.edges[e];
       ptx::fence_proxy_async_smem();
-    } else {
-      // converter warps copy the bucket edges
-      for (int e = tid - 320; e <= p.nl; e += 128) s_edges[e] = p.edges[e];
     }
     ptx::tc_fence_before();
-    ptx::bar_sync_or(6, FC::kThreads - 32, false);   // every warp but the producer
+    ptx::bar_sync_or(kBarSetup, FC::kThreads - 32, false);   // every warp but the producer
     ptx::tc_fence_after();
     tmem = *tmem_holder;
   }
-  const uint32_t tS = tmem, tO = tmem + 2 * N;
-  auto tX = [&](int gq) { return tmem + 6 * N + N * gq; };
+  const uint32_t tS = tmem;                        // S buffer i at +N*i
+  const uint32_t tO = tmem + 2 * N;                // O buffer i at +NP*i
+  auto tX = [&](int gq) { return tmem + 2 * N + 2 * NP + N * gq; };
 
   // ------------------------------------------------------------- producer
   if (warp == 0) {
@@ -207,191 +245,136 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     };
     int bt_cur = bt_load(0);
     int bt_next = bt_load(1);
-    int nchunks = 0, nk = 0, nv = 0;           // chunks, K tiles, V tiles issued
+    int nk = 0, nv = 0, nr = 0;                // K tiles, V tiles, relative chunks issued
     PlanState ps0(p.nl), ps1(p.nl);
     bool ok = true, bad_page = false;
-    int ti = 0;
-    for (; ti < g.ntiles; ++ti) {
+    for (int ti = 0; ti < g.ntiles; ++ti) {
       if (ti > 0 && (ti & 15) == 0) {
         bt_cur = bt_next;
         bt_next = bt_load((ti >> 4) + 1);
       }
       const bool odd = ti & 1;
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, p.edges, odd ? ps1 : ps0);
+      const TilePlan tp = plan_tile<128>(g, ti, p.ex, p.log2_ex, p.log_scale, p.edges, odd ? ps1 : ps0);
       const int c0 = odd ? ps1.c0 : ps0.c0;
+      if (tp.chunk) {
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(rempty(nr % RS), ((nr / RS) & 1) ^ 1, abort_flag, tlim));
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t st = rslot(nr);
+          ptx::mbar_arrive_expect_tx(rfull(nr % RS), FC::kRBytes);
+          ptx::tma_load_3d(st, &p.tmap_r, rfull(nr % RS), 0, c0, h);
+          ptx::tma_load_3d(st + FC::kRHalf, &p.tmap_r, rfull(nr % RS), 64, c0, h);
+        }
+        ++nr;
+      }
       int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
       int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
       if (e0 < 0 || e0 >= p.num_pages) { bad_page = true; e0 = 0; }
       if (tp.npg > 1 && (e1 < 0 || e1 >= p.num_pages)) { bad_page = true; e1 = 0; }
       const int row0 = (e0 * p.Hkv + h) * kPage, row1 = (e1 * p.Hkv + h) * kPage;
-      // E4M3 K tile
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(k8empty(ti % K8S), ((ti / K8S) & 1) ^ 1, abort_flag, tlim));
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(kempty(ti % KS), ((ti / KS) & 1) ^ 1, abort_flag, tlim));
       if (!ok) break;
       if (lane == 0) {
-        const uint32_t st = sbase + FC::oK8 + (ti % K8S) * FC::k8TileBytes;
-        ptx::mbar_arrive_expect_tx(k8full(ti % K8S), tp.npg * FC::k8PageBytes);
-        ptx::tma_load_2d(st, &p.tmap_k, k8full(ti % K8S), 0, row0, pol);
-        if (tp.npg > 1) ptx::tma_load_2d(st + FC::k8PageBytes, &p.tmap_k, k8full(ti % K8S), 0, row1, pol);
+        ptx::mbar_arrive_expect_tx(kfull(ti % KS), tp.npg * FC::kPage8);
+        ptx::tma_load_2d(kslot(ti), &p.tmap_k, kfull(ti % KS), 0, row0, pol);
+        if (tp.npg > 1) ptx::tma_load_2d(kslot(ti) + FC::kPage8, &p.tmap_k, kfull(ti % KS), 0, row1, pol);
       }
       ++nk;
-      // relative-row chunk
-      if (tp.chunk) {
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(xr_empty, (nchunks & 1) ^ 1, abort_flag, tlim));
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t st = sbase + FC::oXR;
-          ptx::mbar_arrive_expect_tx(xr_full, 2 * FC::kRHalfBytes);
-          ptx::tma_load_3d(st, &p.tmap_r, xr_full, 0, c0, h);
-          ptx::tma_load_3d(st + FC::kRHalfBytes, &p.tmap_r, xr_full, 64, c0, h);
-        }
-        ++nchunks;
-      }
-      // E4M3 V tile
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(v8empty(ti % V8S), ((ti / V8S) & 1) ^ 1, abort_flag, tlim));
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(vempty(ti % VS), ((ti / VS) & 1) ^ 1, abort_flag, tlim));
       if (!ok) break;
       if (lane == 0) {
-        const uint32_t st = sbase + FC::oV8 + (ti % V8S) * FC::k8TileBytes;
-        ptx::mbar_arrive_expect_tx(v8full(ti % V8S), tp.npg * FC::k8PageBytes);
-        ptx::tma_load_2d(st, &p.tmap_v, v8full(ti % V8S), 0, row0, pol);
-        if (tp.npg > 1) ptx::tma_load_2d(st + FC::k8PageBytes, &p.tmap_v, v8full(ti % V8S), 0, row1, pol);
+        ptx::mbar_arrive_expect_tx(vfull(ti % VS), tp.npg * FC::kPage8);
+        ptx::tma_load_2d(vslot(ti), &p.tmap_v, vfull(ti % VS), 0, row0, pol);
+        if (tp.npg > 1) ptx::tma_load_2d(vslot(ti) + FC::kPage8, &p.tmap_v, vfull(ti % VS), 0, row1, pol);
       }
       ++nv;
     }
     if (lane == 0) {
       if (bad_page) *bad_page_flag = 1;
-      // Let the copies already issued land before the CTA's memory is
-      // released, on every exit (the consumers may have stopped early).
+      // let the copies already issued land before the CTA's memory is
+      // released, on every exit (the consumers may have stopped early)
       volatile int never = 0;
-      for (int t = max(0, nk - K8S); t < nk; ++t)
-        ptx::mbar_wait(k8full(t % K8S), (t / K8S) & 1, &never, kDrainLimitNs);
-      for (int t = max(0, nv - V8S); t < nv; ++t)
-        ptx::mbar_wait(v8full(t % V8S), (t / V8S) & 1, &never, kDrainLimitNs);
-      if (nchunks > 0) ptx::mbar_wait(xr_full, (nchunks - 1) & 1, &never, kDrainLimitNs);
-    }
-  }
-  // ------------------------------------------------------------ converter
-  // Order K(0), then per tile K(i+1) before V(i): K(i+1) needs only S(i) to
-  // have read the K16 slot, V(i) needs P.V(i-1) to have read the V16 slot,
-  // so the K side runs a tile ahead and S(i+1) and its softmax never wait
-  // behind the P.V chain.
-  else if (warp >= 10) {
-    const int kc = tid - 320;                     // key row of the tile
-    const int sw = kc & 7;
-    // one E4M3 row (128 B, 8 swizzled 16-byte chunks) -> f16 row (two 128 B
-    // halves of the K-major / MN-major 128B-swizzled tile)
-    auto widen = [&](uint32_t src_slot, uint8_t* dst_tile, bool zero) {
-      const uint8_t* src = smem + (src_slot - sbase) + kc * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-        if (!zero) {
-          const uint4 w = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
-          lo4 = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
-                           e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
-          hi4 = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
-                           e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
-        }
-        // 16 dims 16c..16c+15 -> half c/4, 16-byte chunks 2(c%4), 2(c%4)+1
-        uint8_t* row = dst_tile + (c >> 2) * kHalfTileBytes + kc * 128;
-        *reinterpret_cast<uint4*>(row + (((2 * (c & 3)) ^ sw) << 4)) = lo4;
-        *reinterpret_cast<uint4*>(row + (((2 * (c & 3) + 1) ^ sw) << 4)) = hi4;
-      }
-    };
-    auto tile_pages = [&](int ti) { return min(2, g.sp_end - (g.sp_begin + 2 * ti)); };
-    auto convert_k = [&](int ti) -> bool {
-      if (!ptx::mbar_wait(k8full(ti % K8S), (ti / K8S) & 1, abort_flag, tlim) ||
-          !ptx::mbar_wait(kf_empty, (ti & 1) ^ 1, abort_flag, tlim))
-        return false;
-      if (kc < tile_pages(ti) * kPage) widen(sbase + FC::oK8 + (ti % K8S) * FC::k8TileBytes, smem + FC::oKF, false);
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(kf_full);
-      ptx::mbar_arrive(k8empty(ti % K8S));
-      return true;
-    };
-    auto convert_v = [&](int ti) -> bool {
-      // rows no query may see are zeroed: 0 * NaN must not reach P.V
-      const int j = (g.sp_begin + 2 * ti) * kPage + kc;
-      const bool any_valid = kc < tile_pages(ti) * kPage && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
-      if (!ptx::mbar_wait(v8full(ti % V8S), (ti / V8S) & 1, abort_flag, tlim) ||
-          !ptx::mbar_wait(vf_empty, (ti & 1) ^ 1, abort_flag, tlim))
-        return false;
-      widen(sbase + FC::oV8 + (ti % V8S) * FC::k8TileBytes, smem + FC::oVF, !any_valid);
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(vf_full);
-      ptx::mbar_arrive(v8empty(ti % V8S));
-      return true;
-    };
-    bool ok = convert_k(0);
-    for (int ti = 0; ti < g.ntiles && ok; ++ti) {
-      if (ti + 1 < g.ntiles) ok = convert_k(ti + 1);
-      ok = ok && convert_v(ti);
+      for (int t = max(0, nk - KS); t < nk; ++t)
+        ptx::mbar_wait(kfull(t % KS), (t / KS) & 1, &never, kDrainLimitNs);
+      for (int t = max(0, nv - VS); t < nv; ++t)
+        ptx::mbar_wait(vfull(t % VS), (t / VS) & 1, &never, kDrainLimitNs);
+      for (int c = max(0, nr - RS); c < nr; ++c)
+        ptx::mbar_wait(rfull(c % RS), (c / RS) & 1, &never, kDrainLimitNs);
     }
   }
   // ------------------------------------------------------------ MMA issuer
   else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdescQKh = ptx::idesc_f16(128, N, false, false);    // K16 . Qh
-      constexpr uint32_t kIdescXR = ptx::idesc_bf16(128, N, false, false);    // R . Q
-      constexpr uint32_t kIdescPV = ptx::idesc_f16(128, 2 * N, true, true);   // V16^T . P
-      const uint64_t kfdesc = ptx::sdesc_sw128(sbase + FC::oKF, 16, 1024);
-      const uint64_t xrdesc = ptx::sdesc_sw128(sbase + FC::oXR, 16, 1024);
-      const uint64_t qdesc = ptx::sdesc_sw128(sbase + FC::oQ, 16, 1024);
-      const uint64_t qhdesc = ptx::sdesc_sw128(sbase + FC::oQh, 16, 1024);
-      const uint64_t vdesc = ptx::sdesc_sw128(sbase + FC::oVF, kHalfTileBytes, 1024);
-      const uint64_t pdesc = ptx::sdesc_noswz(sbase + FC::oP, 16 * 2 * N, 128);
-      int i = 0, nx = 0;                       // tiles, chunks issued
+      constexpr uint32_t kIdescS = ptx::idesc_e4m3(128, N, false, false);    // K8 . [Q_hi; Q_lo]
+      constexpr uint32_t kIdescPV = ptx::idesc_e4m3(128, NP, true, true);    // V8^T . [P terms]
+      constexpr uint32_t kIdescX = ptx::idesc_bf16(128, N, false, false);    // R . Q
+      const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + FC::oK, 16, 1024);    // K8, K-major
+      const uint64_t q8desc = ptx::sdesc_sw128(sbase + FC::oQ8, 16, 1024);   // Q8, K-major
+      const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + FC::oV, 16, 1024);    // V8^T, MN-major
+      const uint64_t pdesc0 = ptx::sdesc_noswz(sbase + FC::oP, 256, 128);    // P terms, MN-major
+      const uint64_t rdesc0 = ptx::sdesc_sw128(sbase + FC::oR, 16, 1024);    // R chunk, K-major
+      const uint64_t qdesc = ptx::sdesc_sw128(sbase + FC::oQ, 16, 1024);     // bf16 Q, K-major
+      int i = 0, nr = 0;                       // tiles, chunks issued
       int cg[2] = {0, 0};                      // chunks per group
       PlanState ps0(p.nl), ps1(p.nl);
       bool ok = true;
       auto issue_pv = [&](int j) -> bool {
         if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
         if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
-        if (!ptx::mbar_wait(vf_full, j & 1, abort_flag, tlim)) return false;
+        if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
         ptx::tc_fence_after();
-        const uint64_t pbd = pdesc + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
+        const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * FC::kTile8) >> 4);
+        const uint64_t pb = pdesc0 + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
+        // K = 32 keys per MMA: 32 rows of the V tile (4 KB), four 8-key
+        // core-matrix groups of P (1 KB)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::umma_bf16(tO + (j & 1) * 2 * N, vdesc + (uint64_t)((kk * 2048) >> 4),
-                         pbd + (uint64_t)((kk * (2 * 16 * 2 * N)) >> 4), kIdescPV, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_e4m3(tO + (j & 1) * NP, va + (uint64_t)((kk * 4096) >> 4),
+                         pb + (uint64_t)((kk * 1024) >> 4), kIdescPV, kk > 0);
         ptx::umma_commit(o_full + 8u * (j & 1));
-        ptx::umma_commit(vf_empty);
+        ptx::umma_commit(vempty(j % VS));
         return true;
       };
       for (int ti = 0; ti < g.ntiles; ++ti) {
         const int gq = ti & 1;
-        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
-        // S(i) first, then P.V(i-1): the converter widens K(i) before
-        // V(i-1), so S(i) never waits on the P.V chain.
-        const bool pv_pending = i > 0;
+        const TilePlan tp = plan_tile<128>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
+        bool pv_pending = i > 0;
+        if (pv_pending && !ptx::mbar_try_wait(kfull(ti % KS), (ti / KS) & 1)) {
+          if (!(ok = issue_pv(i - 1))) break;
+          pv_pending = false;
+        }
         if (tp.chunk) {
-          ok = ptx::mbar_wait(xr_full, nx & 1, abort_flag, tlim) &&
-               ptx::mbar_wait(x_empty + 8u * gq, (cg[gq] & 1) ^ 1, abort_flag, tlim);
+          const int c = cg[gq];
+          ok = ptx::mbar_wait(rfull(nr % RS), (nr / RS) & 1, abort_flag, tlim) &&
+               ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
           if (!ok) break;
           ptx::tc_fence_after();
+          const uint64_t rd = rdesc0 + (uint64_t)(((nr % RS) * FC::kRBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t ko = (kk >> 2) * FC::kRHalfBytes + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * (N * 128) + (kk & 3) * 32;
-            ptx::umma_bf16(tX(gq), xrdesc + (uint64_t)(ko >> 4), qdesc + (uint64_t)(qo >> 4), kIdescXR, kk > 0);
+            const uint64_t ra = rd + (uint64_t)(((kk >> 2) * FC::kRHalf + (kk & 3) * 32) >> 4);
+            const uint64_t bq = qdesc + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+            ptx::umma_bf16(tX(gq), ra, bq, kIdescX, kk > 0);
           }
           ptx::umma_commit(x_full + 8u * gq);
-          ptx::umma_commit(xr_empty);
-          ++nx;
-          ++cg[gq];
+          ptx::umma_commit(rempty(nr % RS));
+          ++nr;
+          cg[gq] = c + 1;
         }
-        ok = ptx::mbar_wait(kf_full, i & 1, abort_flag, tlim) &&
+        ok = ptx::mbar_wait(kfull(ti % KS), (ti / KS) & 1, abort_flag, tlim) &&
              ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
         if (!ok) break;
         ptx::tc_fence_after();
+        {
+          const uint64_t kd = kdesc0 + (uint64_t)(((ti % KS) * FC::kTile8) >> 4);
+          // K = 32 dims (32 B of each 128 B row) per MMA
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * (N * 128) + (kk & 3) * 32;
-          ptx::umma_bf16(tS + (i & 1) * N, kfdesc + (uint64_t)(ko >> 4), qhdesc + (uint64_t)(qo >> 4),
-                         kIdescQKh, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_e4m3(tS + (i & 1) * N, kd + (uint64_t)((kk * 32) >> 4),
+                           q8desc + (uint64_t)((kk * 32) >> 4), kIdescS, kk > 0);
+          ptx::umma_commit(s_full + 8u * (i & 1));
+          ptx::umma_commit(kempty(ti % KS));
         }
-        ptx::umma_commit(s_full + 8u * (i & 1));
-        ptx::umma_commit(kf_empty);              // the K16 slot is free once S is done
         if (pv_pending && !(ok = issue_pv(i - 1))) break;
         ++i;
       }
@@ -404,7 +387,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   }
   // --------------------------------------------------------------- softmax
   else {
-    constexpr float kLazy = 14.f;             // P = exp2(x - m_ref) < 2^14 stays in f16 range
     const int grp = (warp - 2) >> 2;          // group g takes the tiles i with i % 2 == g
     const int sp = warp & 3;
     const int kl = sp * 32 + lane;            // key lane (S^T) / head-dim lane (O^T)
@@ -415,7 +397,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     float* red = reinterpret_cast<float*>(smem + FC::oRed) + grp * 2 * 4 * FC::kGR;
     const uint32_t tXg = tX(grp) + lane_off;
     const float sl = p.scale_log2;
-    const float ksl = __ldg(p.k_scale + h) * sl;
+    float fq[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) fq[r] = qf[r];
     float l_part[RG], o_acc[RG], m_ref[RG], alpha_r[RG];
 #pragma unroll
     for (int r = 0; r < RG; ++r) { l_part[r] = 0.f; o_acc[r] = 0.f; m_ref[r] = kNoMax; alpha_r[r] = 1.f; }
@@ -423,19 +407,21 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     PlanState ps0(p.nl), ps1(p.nl);
     bool failed = false, aborted = false;
 
+    // O^T of tile j: columns 0..G-1 from P_hi, G..2G-1 from P_mid, 2G..3G-1
+    // from P_lo
     auto process_o = [&](int j) {
-      float ov[8];
+      float ov[24];
       const bool okw = ptx::mbar_wait(o_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        const uint32_t ob = tO + lane_off + (j & 1) * 2 * N;
+        const uint32_t ob = tO + lane_off + (j & 1) * NP;
+        ptx::tmem_ld16(ob, ov);
+        ptx::tmem_ld8(ob + 16, ov + 16);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {          // O^T from P_hi, then from P_lo
-          ptx::tmem_ld8(ob + part * N, ov);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int r = 0; r < RG; ++r) o_acc[r] = part ? o_acc[r] + ov[r] : fmaf(o_acc[r], alpha_r[r], ov[r]);
-        }
+        for (int r = 0; r < RG; ++r)
+          o_acc[r] = fmaf(o_acc[r], alpha_r[r],
+                          ov[r] + fmaf(ov[G + r], 0.0625f, ov[2 * G + r] * 0.00390625f));
         ptx::tc_fence_before();
       }
       ptx::mbar_arrive(o_empty + 8u * (j & 1));
@@ -444,11 +430,11 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 
     for (int ti = 0; ti < g.ntiles; ++ti) {
       const int owner = ti & 1;
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, owner ? ps1 : ps0);
+      const TilePlan tp = plan_tile<128>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, owner ? ps1 : ps0);
       const int c0 = owner ? ps1.c0 : ps0.c0;
       if (owner != grp) continue;
       if (tp.chunk) {
-        // ---- new relative-row chunk: X^T (128 rows x N) -> gather table Y
+        // ---- new relative-row chunk: X^T (128 rows x G) -> gather table Y
         const bool okw = ptx::mbar_wait(x_full + 8u * grp, c & 1, abort_flag, tlim);
         if (okw) {
           float xv[8];
@@ -465,12 +451,12 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       }
       const int i = ti;
 
-      // ---- S^T tile: this thread owns key j
-      float s[8];
+      // ---- S^T tile: this thread owns key j; columns r (Q_hi) and G + r (Q_lo)
+      float sv[16];
       const bool okw = ptx::mbar_wait(s_full + 8u * (i & 1), (i >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
-        ptx::tmem_ld8(tS + lane_off + (i & 1) * N, s);
+        ptx::tmem_ld16(tS + lane_off + (i & 1) * N, sv);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
       }
@@ -490,13 +476,15 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         bk = p.ex + k;
       }
       const float* yrow = Y + (v ? bk - c0 : 0) * YS;
+      float s[RG];
 #pragma unroll
-      for (int r = 0; r < RG; ++r) s[r] = v ? fmaf(s[r], ksl, yrow[r] * sl) : -INFINITY;
+      for (int r = 0; r < RG; ++r)
+        s[r] = v ? fmaf(fmaf(sv[G + r], 0.0625f, sv[r]), fq[r], yrow[r] * sl) : -INFINITY;
 
-      // ---- lazy max (as the bf16 kernel, threshold 2^14)
+      // ---- lazy max (threshold 2^8: P stays inside E4M3 range)
       bool over = false;
 #pragma unroll
-      for (int r = 0; r < RG; ++r) over |= s[r] > m_ref[r] + kLazy;
+      for (int r = 0; r < RG; ++r) over |= s[r] > m_ref[r] + kLazy8;
       if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, over || !okw || failed)) {
         if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
         float* redb = red + (li & 1) * 4 * FC::kGR;
@@ -519,27 +507,58 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int r = 0; r < RG; ++r) alpha_r[r] = 1.f;
       }
-      // ---- P = exp2(x - m_ref) as f16 hi + lo parts, stacked [P_hi; P_lo],
-      //      MN-major without swizzle (8-row x 16-byte core matrices)
+      // ---- P = exp2(x - m_ref) in [0, 2^8] as P_hi + P_mid / 16 + P_lo / 256
+      //      (each the E4M3 code of 2^(4k) x what the earlier terms left;
+      //      the remainders are exact in fp32), one 32-byte row per key:
+      //      bytes 0..G-1 P_hi, G..2G-1 P_mid, 2G..3G-1 P_lo, the rest zero;
+      //      MN-major without swizzle (8-key x 16-byte core matrices, 8-key
+      //      groups 256 B apart, the two 16-row halves 128 B apart)
       {
-        const uint32_t pbuf = sbase + FC::oP + (uint32_t)((i & 1) * FC::kPBufBytes);
-        const uint32_t prow = pbuf + (uint32_t)((kl >> 3) * (16 * 2 * N) + (kl & 7) * 16);
-        uint32_t hi[4], lo[4];
+        uint32_t hi[RG / 2], mid[RG / 2], low[RG / 2];
 #pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
+        for (int q2 = 0; q2 < RG / 2; ++q2) {
           const int r0 = 2 * q2, r1 = r0 + 1;
-          float p0 = 0.f, p1 = 0.f;
-          if (r0 < RG) { p0 = exp2f(s[r0] - m_ref[r0]); l_part[r0] += p0; }
-          if (r1 < RG) { p1 = exp2f(s[r1] - m_ref[r1]); l_part[r1] += p1; }
-          const __half2 h2 = __floats2half2_rn(p0, p1);
-          const __half2 l2 = __floats2half2_rn(p0 - __low2float(h2), p1 - __high2float(h2));
-          hi[q2] = *reinterpret_cast<const uint32_t*>(&h2);
-          lo[q2] = *reinterpret_cast<const uint32_t*>(&l2);
+          const float p0 = exp2f(s[r0] - m_ref[r0]), p1 = exp2f(s[r1] - m_ref[r1]);
+          l_part[r0] += p0;
+          l_part[r1] += p1;
+          hi[q2] = e4m3x2_rn(p0, p1);
+          const float2 vh = e4m3x2_value(hi[q2]);
+          const float a0 = p0 - vh.x, a1 = p1 - vh.y;
+          mid[q2] = e4m3x2_rn(a0 * 16.f, a1 * 16.f);
+          const float2 vm = e4m3x2_value(mid[q2]);
+          low[q2] = e4m3x2_rn(fmaf(vm.x, -0.0625f, a0) * 256.f, fmaf(vm.y, -0.0625f, a1) * 256.f);
         }
+        // the row of bytes [hi | mid | lo | 0...] as 8 little-endian words
+        uint32_t w[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) w[q] = 0u;
+#pragma unroll
+        for (int q2 = 0; q2 < RG / 2; ++q2) {
+          const int bh = 2 * q2, bm = G + 2 * q2, bl = 2 * G + 2 * q2;   // byte offsets
+          w[bh >> 2] |= hi[q2] << ((bh & 3) * 8);
+          w[bm >> 2] |= mid[q2] << ((bm & 3) * 8);
+          w[bl >> 2] |= low[q2] << ((bl & 3) * 8);
+        }
+        const uint32_t prow = sbase + FC::oP + (uint32_t)((i & 1) * FC::kPBufBytes) +
+                              (uint32_t)((kl >> 3) * 256 + (kl & 7) * 16);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                     ::"r"(prow), "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
+                     ::"r"(prow), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                     ::"r"(prow + N * 16), "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
+                     ::"r"(prow + 128), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]) : "memory");
+      }
+      // ---- keys no token may see: clear their V rows (stale or poisoned
+      //      codes must not reach P.V, where 0 * NaN = NaN)
+      {
+        const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
+        if (!any_valid) {
+          if (ptx::mbar_wait(vfull(i % VS), (i / VS) & 1, abort_flag, tlim)) {
+            uint4* vrow = reinterpret_cast<uint4*>(smem + FC::oV + (i % VS) * FC::kTile8 + kl * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) vrow[q] = make_uint4(0, 0, 0, 0);
+          } else {
+            failed = true;
+          }
+        }
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
@@ -549,8 +568,8 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     ptx::pdl_launch_dependents();
 
     // ---- epilogue: the two groups hold the same rows; merge them by LSE
-    //      through the idle staging ring, scale by the V scale, write
-    bool bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, aborted || failed);
+    //      through the idle K ring, scale by the V scale, write
+    bool bad = ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, aborted || failed);
     float* eo = reinterpret_cast<float*>(smem);             // [NG][RG][128]
     float* el = eo + NG * RG * kHeadDim;                    // [NG][RG][128]
     float* em = el + NG * RG * kHeadDim;                    // [NG][RG]
@@ -566,7 +585,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         for (int r = 0; r < RG; ++r) em[grp * RG + r] = m_ref[r];
       }
     }
-    bad = ptx::bar_sync_or(3, kSoftmaxThreads * NG, bad);
+    bad = ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, bad);
     if (!bad) {
       const int et = tid - 64, ew = et >> 5;
       for (int q = ew; q < NG * RG; q += 4 * NG) {
@@ -574,10 +593,10 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         const float vsum = warp_sum(src[lane] + src[lane + 32] + src[lane + 64] + src[lane + 96]);
         if (lane == 0) es[q] = vsum;
       }
-      ptx::bar_sync_or(3, kSoftmaxThreads * NG, false);
+      ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, false);
       const float vsc = __ldg(p.v_scale + h);
       const int rows = p.B * p.Hq;
-      for (int e = et; e < NQ * kHeadDim; e += kSoftmaxThreads * NG) {
+      for (int e = et; e < RG * kHeadDim; e += kSoftmaxThreads * NG) {
         const int n = e / kHeadDim, dd = e % kHeadDim;
         const float m = fmaxf(em[n], em[RG + n]);
         const float sc0 = exp2f(em[n] - m), sc1 = exp2f(em[RG + n] - m);

@@ -132,8 +132,8 @@ def test_supported_group_shapes(ra, kw):
     assert ra.rel_attn_workspace_bytes(s, 3) == 256 + (3 * rows * 4 + 255) // 256 * 256 + 3 * rows * 128 * 4
 
 
-def test_e4m3_only_for_48_over_8(ra):
-    s = shape(ra, num_q_heads=64, num_kv_heads=8)
+def test_e4m3_only_for_one_token(ra):
+    s = shape(ra, num_q_heads=64, num_kv_heads=8, q_tokens=2)
     fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
     rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
                                      fake, 0, 1, fake, None, fake, 1 << 30, None)

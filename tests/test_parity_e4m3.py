@@ -1,7 +1,8 @@
 """GPU parity of the E4M3 (FP8) KV-cache path against the fp64 oracle.
 
 The oracle dequantises the codes exactly (code value x per-KV-head scale) and
-applies the definition; the kernel widens the codes to f16 on chip.  Same
+applies the definition; the kernel runs the codes through E4M3 tensor-core
+MMAs, with the query split into two E4M3 terms and P into three.  Same
 tolerances as the bf16 path: max |out_fp32 - oracle| <= 2e-3, max |lse -
 oracle| <= 1e-3.
 """
@@ -60,9 +61,9 @@ def check(out, lse, ref_out, ref_lse):
     assert eo <= OUT_TOL and el <= LSE_TOL, (eo, el)
 
 
-def small(L, window=0, NB=1280, seed=0, Hkv=2, lens=None, **kw):
+def small(L, window=0, NB=1280, seed=0, Hkv=2, lens=None, G=6, **kw):
     lens = lens if lens is not None else [L]
-    return W.make_case(seq_lens=lens, q_tokens=1, num_q_heads=6 * Hkv, num_kv_heads=Hkv,
+    return W.make_case(seq_lens=lens, q_tokens=1, num_q_heads=G * Hkv, num_kv_heads=Hkv,
                        window=window, num_buckets=NB, seed=seed, extra_pages=2, **kw).to("cuda")
 
 
@@ -72,6 +73,9 @@ SMALL = [
     dict(L=1500, window=1), dict(L=1500, window=64), dict(L=2500, window=1024),
     dict(L=900, NB=8), dict(L=2000, NB=1030), dict(L=200, window=1024, NB=1024),
     dict(L=6000, NB=364, exact_buckets=64, max_distance=5000),
+    # the previous Inkling's group sizes
+    dict(L=1, G=4), dict(L=129, G=4), dict(L=3001, G=4), dict(L=2500, G=4, window=512, NB=1024),
+    dict(L=1, G=8), dict(L=129, G=8), dict(L=3001, G=8), dict(L=5000, G=8, seed=5),
 ]
 
 
@@ -159,6 +163,75 @@ def test_sliding_100k(ra):
     ref = run_oracle(case, codes)
     for s in (1, 4, 0):
         check(*run_gpu(ra, case, codes, s), *ref)
+
+
+def test_one_hot_key_probe(ra):
+    """One key dominates its row (P = 1 there, tiny elsewhere): the hardest
+    case for the three-term split of P, whose largest term then carries
+    almost all of the output."""
+    for j_star in (0, 64, 500, 999):
+        case = small(1000, Hkv=1)
+        case.rel_table.zero_()
+        q = case.q[0, 0, 0].float()
+        pg = int(case.block_table[0, j_star // 64])
+        case.k_cache[pg, 0, j_star % 64] = (q * (40.0 / q.norm())).to(torch.bfloat16)
+        codes = e4m3(case)
+        check(*run_gpu(ra, case, codes, 0), *run_oracle(case, codes))
+
+
+def test_query_magnitudes(ra):
+    """Query rows of very different scales (1e-3 .. 30) and a row with tiny
+    elements among large ones: the per-row power of two and the two-term
+    E4M3 split of the query keep q . k exact."""
+    case = small(2000, Hkv=2)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    scale = torch.tensor([1e-3, 0.05, 1.0, 3.0, 30.0, 0.3] * 2, device="cuda")
+    case.q.copy_((case.q.float() * scale[None, None, :, None]).to(torch.bfloat16))
+    case.q[0, 0, 3, ::2] = (torch.randn(64, generator=g, device="cuda") * 1e-4).to(torch.bfloat16)
+    codes = e4m3(case)
+    check(*run_gpu(ra, case, codes, 3), *run_oracle(case, codes))
+
+
+@pytest.mark.parametrize("name", ["v1_full_100k"])
+def test_previous_model_full_layer(ra, name):
+    case = W.make_workload(name, seed=0, device="cuda")
+    codes = e4m3(case)
+    ref = run_oracle(case, codes)
+    for s in (1, 18, 0):
+        check(*run_gpu(ra, case, codes, s), *ref)
+
+
+def test_injected_wait_limit_times_out_cleanly(ra):
+    """As for the bf16 kernel: a 1 us wait bound makes the E4M3 kernel abort
+    promptly with TIMEOUT and NaN rows; the default bound then works again."""
+    import time
+    case = W.make_workload("full_100k", seed=4, device="cuda", num_q_heads=12, num_kv_heads=2)
+    codes = e4m3(case)
+    shape = ra.shape_of(case.q, codes[0], case.block_table, case.rel_table,
+                        max_seq_len=case.max_seq_len, out_fp32=True)
+    ws = ra.Workspace.for_shape(shape, 0, "cuda")
+    kc, vc, ks, vs = codes
+    call = lambda: ra.rel_attn_decode_e4m3(case.q, kc, vc, ks, vs, case.block_table, case.seq_lens,
+                                           case.rel_table, 0, 0, workspace=ws,
+                                           max_seq_len=case.max_seq_len, out_fp32=True)
+    call()
+    torch.cuda.synchronize()
+    assert ws.read_status() == ra.REL_ATTN_OK
+    try:
+        ra.rel_attn_set_wait_limit(1000)
+        t0 = time.perf_counter()
+        out, lse = call()
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        ra.rel_attn_set_wait_limit(0)
+    assert elapsed < 1.0
+    assert ws.read_status() == ra.REL_ATTN_ERR_TIMEOUT
+    assert torch.isnan(out).any()
+    out, lse = call()
+    torch.cuda.synchronize()
+    check(out, lse, *run_oracle(case, codes))
+    assert ws.read_status() == ra.REL_ATTN_OK
 
 
 def test_rejects_several_query_tokens_and_missing_scales(ra):
