@@ -209,6 +209,34 @@ int rel_attn_decode_static(const rel_attn_shape* shape, const void* q,
                            void* out, float* lse, void* stream);
 
 /*
+ * rel_attn_prefill -- the same attention for many query tokens per
+ * sequence at once: a prefill, or a chunk of one ("vLLM、Inkling 2 Smallを
+ * 初日サポート GB200で630 tok/s", section "vLLMの最適化と性能", and
+ * "A vLLM már az első napon támogatja a Reflection Beam modellt" measure
+ * 8K-token and 8 x 2,048-token prefills).  Query token t of sequence b sits
+ * at position L_b - C + t and attends causally (and within the window) to
+ * every key up to it, exactly as the tokens of a decode step do.
+ *
+ *   shape       as for rel_attn_decode except q_tokens = C, the query tokens
+ *               per sequence, 1 .. 2^20 (batch * ceil(C / 8) <= 65535).
+ *   q, out      [B, C, Hq, D]; lse [B, C, Hq] or NULL.
+ *   seq_lens    L_b, counting the C query tokens (C <= L_b).
+ *   workspace   rel_attn_workspace_bytes(shape, num_splits) bytes with this
+ *               shape (q_tokens = C); num_splits <= 0 picks one split per
+ *               chunk unless the chunks are too few to fill the GPU.
+ * Every other argument, the error handling and the status word are as for
+ * rel_attn_decode.  The tokens run as chunks of 8 through the decode
+ * kernels (the first C mod 8 tokens as one more chunk), each chunk reading
+ * the keys up to its last token.
+ */
+int rel_attn_prefill(const rel_attn_shape* shape, const void* q,
+                     const void* k_cache, const void* v_cache,
+                     const int32_t* block_table, const int32_t* seq_lens,
+                     const void* rel_table, int window, int num_splits,
+                     void* out, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
  * rel_attn_kv_write -- the producer step that fills the cache the decode
  * reads: a short convolution over the new tokens' K and V, written into the
  * paged KV cache (bf16, or E4M3 codes), with the raw K/V kept for the next

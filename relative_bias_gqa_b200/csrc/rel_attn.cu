@@ -488,6 +488,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const unsigned long long wl = g_wait_limit_ns.load(std::memory_order_relaxed);
   prm->timeout_ns = wl ? wl : kDefaultTimeoutNs;
   prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
+  prm->cps = 1; prm->seq_stride = T; prm->tok_off = 0; prm->len_off = 0;
+  prm->rows_total = (int)rows;
   prm->num_pages = shape->num_pages;
   prm->max_pages = shape->max_pages_per_seq;
   prm->num_splits = S;
@@ -648,6 +650,96 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out, flo
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Chunked prefill: the C query tokens of each sequence run as chunks of
+// kPrefillChunk tokens through the multi-token decode instances (each chunk a
+// virtual batch entry on its sequence's block-table row, attending causally
+// to everything before it), the first C % kPrefillChunk tokens as one more
+// launch of the instance for that many tokens; then the combine kernel when
+// the keys are split.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kPrefillChunk = 8;
+}  // namespace
+
+extern "C" int rel_attn_prefill(const rel_attn_shape* shape, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_table,
+                                const int32_t* seq_lens, const void* rel_table, int window,
+                                int num_splits, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!shape) return REL_ATTN_ERR_INVALID_ARG;
+  const int C = shape->q_tokens;
+  if (C < 1 || C > (1 << 20)) return REL_ATTN_ERR_INVALID_ARG;
+  // validate everything else as for a decode step of one chunk (never more
+  // rows than the whole prefill, so its workspace check is implied by ours)
+  const int nfull = C / kPrefillChunk, rem = C % kPrefillChunk;
+  rel_attn_shape chunk_shape = *shape;
+  chunk_shape.q_tokens = nfull > 0 ? kPrefillChunk : rem;
+  int rc = validate_shape(&chunk_shape);
+  if (rc != REL_ATTN_OK) return rc;
+  if ((long long)shape->batch * (nfull > 0 ? nfull : 1) > 65535) return REL_ATTN_ERR_INVALID_ARG;
+  if (num_splits > 256) return REL_ATTN_ERR_INVALID_ARG;
+  int dev;
+  rc = probe_device(&dev);
+  if (rc != REL_ATTN_OK) return rc;
+  // one split per chunk unless the chunks do not fill the GPU
+  int S = num_splits;
+  if (S <= 0) {
+    const long long units = (long long)shape->batch * shape->num_kv_heads * (nfull + (rem > 0));
+    S = (units >= g_dev[dev].sm_count) ? 1 : (int)std::max<long long>(1, g_dev[dev].sm_count / units);
+    const long long cap = (long long)shape->max_pages_per_seq * kPage;
+    const long long len = shape->max_seq_len > 0 ? std::min<long long>(shape->max_seq_len, cap) : cap;
+    S = (int)std::max<long long>(1, std::min<long long>(S, (len + 2 * kPage - 1) / (2 * kPage)));
+  }
+  // `shape` (q_tokens = C) sizes the workspace: all B * C * Hq rows' partials
+  DecodeParams prm;
+  int S_used = 0;
+  DeviceInfo* di = nullptr;
+  rc = prepare(&chunk_shape, q, k_cache, v_cache, block_table, seq_lens, rel_table, window, S,
+               out, lse, workspace, workspace_bytes, &prm, &S_used, &di);
+  if (rc != REL_ATTN_OK) return rc;
+  const size_t rows = (size_t)shape->batch * C * shape->num_q_heads;
+  if (workspace_bytes < workspace_for(shape, S)) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  prm.ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes);
+  prm.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
+  prm.rows_total = (int)rows;
+  prm.seq_stride = C;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = shape->batch, Hkv = shape->num_kv_heads, G = shape->num_q_heads / Hkv;
+  if (nfull > 0) {
+    DecodeParams pf = prm;
+    pf.T = kPrefillChunk;
+    pf.cps = nfull;
+    pf.tok_off = rem;
+    pf.len_off = 0;
+    if (!cached_map(&pf.tmap_r, group_width_for(G, kPrefillChunk) == 16 ? 3 : 2, rel_table,
+                    (uint64_t)shape->num_buckets, (uint64_t)Hkv))
+      return REL_ATTN_ERR_CUDA;
+    rel_attn_shape sh = chunk_shape;
+    sh.batch = B * nfull;
+    sh.q_tokens = kPrefillChunk;
+    rc = launch_partial_any(pf, &sh, S, st, *di);
+    if (rc != REL_ATTN_OK) return rc;
+  }
+  if (rem > 0) {
+    DecodeParams pr = prm;
+    pr.T = rem;
+    pr.cps = 1;
+    pr.tok_off = 0;
+    pr.len_off = C - rem;
+    if (!cached_map(&pr.tmap_r, group_width_for(G, rem) == 16 ? 3 : 2, rel_table,
+                    (uint64_t)shape->num_buckets, (uint64_t)Hkv))
+      return REL_ATTN_ERR_CUDA;
+    rel_attn_shape sh = chunk_shape;
+    sh.q_tokens = rem;
+    rc = launch_partial_any(pr, &sh, S, st, *di);
+    if (rc != REL_ATTN_OK) return rc;
+  }
+  if (S == 1) return REL_ATTN_OK;
+  return launch_combine(shape, S, out, lse, workspace, st);
+}
 
 // ---------------------------------------------------------------------------
 // The KV-cache producer step: short convolution over the new tokens' K and V,

@@ -104,7 +104,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   g.T = T;
   if (g.L < T || g.L > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
-    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     return;
   }
   g.p0 = g.L - T;
@@ -113,7 +113,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, &g.sp_begin, &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {
-    fill_rows<G>(p, b, h, s_idx, 0.f, -INFINITY);
+    fill_rows<G>(p, first_token_row(p, b), h, s_idx, 0.f, -INFINITY);
     return;
   }
 
@@ -595,7 +595,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, false);
       const float vsc = __ldg(p.v_scale + h);
-      const int rows = p.B * p.Hq;
+      const int rows = p.rows_total;
       for (int e = et; e < RG * kHeadDim; e += kSoftmaxThreads * NG) {
         const int n = e / kHeadDim, dd = e % kHeadDim;
         const float m = fmaxf(em[n], em[RG + n]);
@@ -628,7 +628,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     if (bad_cta) atomicOr(p.status, kStatusBadSeq);
   }
   if (aborted_cta || bad_cta)
-    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);

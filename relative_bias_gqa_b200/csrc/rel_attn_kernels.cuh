@@ -93,6 +93,15 @@ struct alignas(64) DecodeParams {
   unsigned* status;
   unsigned long long timeout_ns;
   int B, T, Hq, Hkv, num_pages, max_pages, num_splits, window, out_fp32;
+  // Row mapping.  Grid z-index b is chunk (b % cps) of sequence (b / cps);
+  // its T query tokens are rows tok(b) .. tok(b) + T - 1 of q / out / lse
+  // (rows of Hq heads), tok(b) = (b / cps) * seq_stride + tok_off +
+  // (b % cps) * T, and its context length is seq_lens[b / cps] - len_off -
+  // (cps - 1 - b % cps) * T.  A decode step is cps = 1, seq_stride = T,
+  // tok_off = len_off = 0; a chunked prefill runs cps chunks of T tokens of
+  // one sequence, each attending causally to everything before it.
+  int cps, seq_stride, tok_off, len_off;
+  int rows_total;       // rows of the partial buffers: all query tokens x Hq
   int ex;               // distances d < ex are their own bucket
   int nl;               // tail buckets: bucket = ex + max{k < nl : edges[k] <= d}
   float scale_log2;     // log2(e) / sqrt(D)
@@ -362,16 +371,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// First query-token row of grid z-index b (see DecodeParams).
+__device__ __forceinline__ int first_token_row(const DecodeParams& p, int b) {
+  const int bs = b / p.cps;
+  return bs * p.seq_stride + p.tok_off + (b - bs * p.cps) * p.T;
+}
+// Context length of grid z-index b's query chunk, given its sequence's
+// length L_seq.
+__device__ __forceinline__ int chunk_seq_len(const DecodeParams& p, int b, int L_seq) {
+  const int bs = b / p.cps;
+  return L_seq - p.len_off - (p.cps - 1 - (b - bs * p.cps)) * p.T;
+}
+
 // Write this CTA's rows (all NQ rows of the group, every head-dim) with a
-// constant value; used for empty splits and rejected sequences.
+// constant value; used for empty splits and rejected sequences.  tok0 =
+// the first query token's row.
 template <int G>
-__device__ void fill_rows(const DecodeParams& p, int b, int h, int s, float o_val, float lse_val) {
-  const int rows = p.B * p.T * p.Hq;
+__device__ void fill_rows(const DecodeParams& p, int tok0, int h, int s, float o_val, float lse_val) {
+  const int rows = p.rows_total;
   const int NQ = p.T * G;
   for (int e = threadIdx.x; e < NQ * kHeadDim; e += blockDim.x) {
     const int n = e / kHeadDim, d = e % kHeadDim;
     const int t = n / G, gg = n % G;
-    const int row = (b * p.T + t) * p.Hq + h * G + gg;
+    const int row = (tok0 + t) * p.Hq + h * G + gg;
     if (p.num_splits == 1) {
       if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o_val;
       else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o_val);
@@ -416,12 +438,17 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
                                                    RG <= KC::kGR), "group width");
 
   // ------------------------------------------------------------ geometry
+  const int tok0 = first_token_row(p, b);      // row of query token 0
+  const int b_seq = b / p.cps;                 // the sequence (block-table row)
   SplitGeom g;
-  g.L = __ldg(p.seq_lens + b);
+  // the sequence must hold all of its query tokens (seq_stride of them: T
+  // for a decode step, C for a prefill) and fit its block-table row
+  const int L_seq = __ldg(p.seq_lens + b_seq);
+  g.L = chunk_seq_len(p, b, L_seq);
   g.T = T;
-  if (g.L < T || g.L > p.max_pages * kPage) {
+  if (L_seq < p.seq_stride || L_seq > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
-    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, tok0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     return;
   }
   g.p0 = g.L - T;
@@ -430,7 +457,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, &g.sp_begin, &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {                       // a trailing split with no page
-    fill_rows<G>(p, b, h, s_idx, 0.f, -INFINITY);
+    fill_rows<G>(p, tok0, h, s_idx, 0.f, -INFINITY);
     return;
   }
 
@@ -518,7 +545,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
         if (nl >= 0) {
           const int t = nl / G, gg = nl % G;
-          const __nv_bfloat16* src = p.q + ((size_t)(b * T + t) * p.Hq + h * G + gg) * kHeadDim
+          const __nv_bfloat16* src = p.q + ((size_t)(tok0 + t) * p.Hq + h * G + gg) * kHeadDim
                                      + half * 64 + w16 * 8;
           v = __ldg(reinterpret_cast<const uint4*>(src));
         }
@@ -539,7 +566,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   // ------------------------------------------------------------- producer
   if (warp == 0) {
     const uint64_t pol = ptx::l2_policy_evict_first();
-    const int* bt_row = p.block_table + (size_t)b * p.max_pages;
+    const int* bt_row = p.block_table + (size_t)b_seq * p.max_pages;
     auto bt_load = [&](int grp) -> int {
       const int pg = g.sp_begin + 32 * grp + lane;
       return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
@@ -1045,7 +1072,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (lane == 0) es[q] = v;
       }
       ptx::bar_sync_or(kBarSoftmaxAll, kSoftmaxThreads * NG, false);
-      const int rows = p.B * T * p.Hq;
+      const int rows = p.rows_total;
       // output rows: (token t, head gg) <- entries (group, local row)
       for (int e = et; e < NQ * kHeadDim; e += kSoftmaxThreads * NG) {
         const int n = e / kHeadDim, d = e % kHeadDim;
@@ -1077,7 +1104,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
         o = (l > 0.f) ? o / l : 0.f;
         const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int row = (b * T + t) * p.Hq + h * G + gg;
+        const int row = (tok0 + t) * p.Hq + h * G + gg;
         if (p.num_splits == 1) {
           if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
           else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
@@ -1104,7 +1131,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     if (bad_cta) atomicOr(p.status, kStatusBadSeq);
   }
   if (aborted_cta || bad_cta)
-    fill_rows<G>(p, b, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, tok0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, KC::kTmemCols);

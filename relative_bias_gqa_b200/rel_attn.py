@@ -28,7 +28,7 @@ EXPORTED = (
     "rel_attn_read_status", "rel_attn_choose_splits", "rel_attn_bucket",
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
     "rel_attn_split_pages", "rel_attn_decode_e4m3", "rel_attn_partial_e4m3",
-    "rel_attn_set_wait_limit", "rel_attn_kv_write",
+    "rel_attn_set_wait_limit", "rel_attn_kv_write", "rel_attn_prefill",
 )
 
 
@@ -79,6 +79,8 @@ def _load():
     lib.rel_attn_split_pages.argtypes = [SP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.rel_attn_split_pages.restype = ctypes.c_int
+    lib.rel_attn_prefill.argtypes = lib.rel_attn_decode.argtypes
+    lib.rel_attn_prefill.restype = ctypes.c_int
     lib.rel_attn_kv_write.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.rel_attn_kv_write.restype = ctypes.c_int
     lib.rel_attn_set_wait_limit.argtypes = [ctypes.c_ulonglong]
@@ -255,6 +257,50 @@ def rel_attn_decode_e4m3(q, k_codes, v_codes, k_scale, v_scale, block_table, seq
     if rc != REL_ATTN_OK:
         raise RelAttnError(rc)
     return out, lse
+
+
+def rel_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, rel_table, window: int = 0,
+                     num_splits: int = 0, out=None, lse=None, workspace: Optional[Workspace] = None,
+                     *, max_seq_len: int = 0, out_fp32: bool = False, exact_buckets: int = 1024,
+                     max_distance: int = 1 << 20, stream=None, with_lse: bool = True):
+    """Attention for all C query tokens of each sequence (q [B, C, Hq, D],
+    token t at position seq_len - C + t, causal); arguments as for
+    rel_attn_decode.  Returns (out, lse)."""
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
+                        ("v_cache", v_cache, torch.bfloat16), ("rel_table", rel_table, torch.bfloat16),
+                        ("block_table", block_table, torch.int32), ("seq_lens", seq_lens, torch.int32)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    shape = shape_of(q, k_cache, block_table, rel_table, max_seq_len=max_seq_len,
+                     out_fp32=out_fp32, exact_buckets=exact_buckets, max_distance=max_distance)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = prefill_workspace_bytes(shape, num_splits)
+        workspace = Workspace(n, q.device)
+    rc = lib.rel_attn_prefill(
+        ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        block_table.data_ptr(), seq_lens.data_ptr(), rel_table.data_ptr(),
+        int(window), int(num_splits), out.data_ptr(),
+        lse.data_ptr() if lse is not None else None,
+        workspace.buf.data_ptr(), workspace.nbytes, _stream_ptr(stream))
+    if rc != REL_ATTN_OK:
+        raise RelAttnError(rc)
+    return out, lse
+
+
+def prefill_workspace_bytes(shape: RelAttnShape, num_splits: int) -> int:
+    """Workspace bytes rel_attn_prefill needs: the status word, plus, with
+    more than one split, every row's partials (the layout of the decode
+    workspace for B * C rows).  num_splits <= 0 assumes up to 256."""
+    S = num_splits if num_splits > 0 else 256
+    rows = shape.batch * shape.q_tokens * shape.num_q_heads
+    if S == 1:
+        return 256
+    return 256 + (S * rows * 4 + 255) // 256 * 256 + S * rows * 128 * 4
 
 
 def rel_attn_kv_write(k_new, v_new, conv_w, k_raw, v_raw, k_cache, v_cache, block_table,
