@@ -438,7 +438,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
                                                    RG <= KC::kGR), "group width");
 
   // ------------------------------------------------------------ geometry
-  const int tok0 = first_token_row(p, b);      // row of query token 0
+  const int row0 = first_token_row(p, b);      // q / out row of query token 0
   const int b_seq = b / p.cps;                 // the sequence (block-table row)
   SplitGeom g;
   // the sequence must hold all of its query tokens (seq_stride of them: T
@@ -448,7 +448,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   g.T = T;
   if (L_seq < p.seq_stride || L_seq > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
-    fill_rows<G>(p, tok0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, row0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     return;
   }
   g.p0 = g.L - T;
@@ -457,7 +457,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, &g.sp_begin, &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {                       // a trailing split with no page
-    fill_rows<G>(p, tok0, h, s_idx, 0.f, -INFINITY);
+    fill_rows<G>(p, row0, h, s_idx, 0.f, -INFINITY);
     return;
   }
 
@@ -545,7 +545,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
         if (nl >= 0) {
           const int t = nl / G, gg = nl % G;
-          const __nv_bfloat16* src = p.q + ((size_t)(tok0 + t) * p.Hq + h * G + gg) * kHeadDim
+          const __nv_bfloat16* src = p.q + ((size_t)(row0 + t) * p.Hq + h * G + gg) * kHeadDim
                                      + half * 64 + w16 * 8;
           v = __ldg(reinterpret_cast<const uint4*>(src));
         }
@@ -1104,7 +1104,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
         o = (l > 0.f) ? o / l : 0.f;
         const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int row = (tok0 + t) * p.Hq + h * G + gg;
+        const int row = (row0 + t) * p.Hq + h * G + gg;
         if (p.num_splits == 1) {
           if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + d] = o;
           else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + d] = __float2bfloat16_rn(o);
@@ -1131,7 +1131,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     if (bad_cta) atomicOr(p.status, kStatusBadSeq);
   }
   if (aborted_cta || bad_cta)
-    fill_rows<G>(p, tok0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, row0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, KC::kTmemCols);
