@@ -56,8 +56,9 @@ struct Fp8Config {
   // kfull/kempty[KS] vfull/vempty[VS] rfull/rempty[RS] s_full/s_empty[2]
   // p_full[2] o_full/o_empty[2] x_full/x_empty[2] drain
   static constexpr int kNumBars = 2 * (kKSlots + kVSlots + kRSlots) + 4 + 2 + 4 + 4 + 1;
-  static constexpr int oMisc = oBar + kNumBars * 8;             // tmem base, abort, bad page
-  static constexpr int kBytes = oMisc + 16;
+  // tmem base, abort flag, bad-page flag, K / V tiles and relative chunks issued
+  static constexpr int oMisc = oBar + kNumBars * 8;
+  static constexpr int kBytes = oMisc + 32;
   static constexpr int kAllocBytes = kBytes + 1024;
   static constexpr int kTmemCols = 128;                         // S[2] 32 + O[2] 64 + X[2] 32
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
@@ -105,6 +106,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   if (g.L < T || g.L > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
     fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    finish_split<G>(p, b, h, first_token_row(p, b));
     return;
   }
   g.p0 = g.L - T;
@@ -114,6 +116,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {
     fill_rows<G>(p, first_token_row(p, b), h, s_idx, 0.f, -INFINITY);
+    finish_split<G>(p, b, h, first_token_row(p, b));
     return;
   }
 
@@ -139,6 +142,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + FC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 4);
   volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 8);
+  int* issued = reinterpret_cast<int*>(smem + FC::oMisc + 12);   // [K tiles, V tiles, chunks]
   auto kslot = [&](int i) { return sbase + FC::oK + (uint32_t)((i % KS) * FC::kTile8); };
   auto vslot = [&](int i) { return sbase + FC::oV + (uint32_t)((i % VS) * FC::kTile8); };
   auto rslot = [&](int c) { return sbase + FC::oR + (uint32_t)((c % RS) * FC::kRBytes); };
@@ -161,6 +165,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *bad_page_flag = 0;
+    issued[0] = issued[1] = issued[2] = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&p.tmap_k);
     ptx::prefetch_tmap(&p.tmap_v);
@@ -291,15 +296,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     }
     if (lane == 0) {
       if (bad_page) *bad_page_flag = 1;
-      // let the copies already issued land before the CTA's memory is
-      // released, on every exit (the consumers may have stopped early)
-      volatile int never = 0;
-      for (int t = max(0, nk - KS); t < nk; ++t)
-        ptx::mbar_wait(kfull(t % KS), (t / KS) & 1, &never, kDrainLimitNs);
-      for (int t = max(0, nv - VS); t < nv; ++t)
-        ptx::mbar_wait(vfull(t % VS), (t / VS) & 1, &never, kDrainLimitNs);
-      for (int c = max(0, nr - RS); c < nr; ++c)
-        ptx::mbar_wait(rfull(c % RS), (c / RS) & 1, &never, kDrainLimitNs);
+      issued[0] = nk;                        // for the drain at teardown
+      issued[1] = nv;
+      issued[2] = nr;
     }
   }
   // ------------------------------------------------------------ MMA issuer
@@ -624,7 +623,19 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   // writes its rows as NaN (see the bf16 kernel)
   const bool aborted_cta = *abort_flag != 0, bad_cta = *bad_page_flag != 0;
   if (tid == 0) {
-    if (aborted_cta) atomicOr(p.status, kStatusTimeout);
+    if (aborted_cta) {
+      atomicOr(p.status, kStatusTimeout);
+      // the consumers stopped early: let the copies already issued land
+      // before the CTA's memory is released (see the bf16 kernel)
+      volatile int never = 0;
+      const int nk = issued[0], nv = issued[1], nr = issued[2];
+      for (int t = max(0, nk - KS); t < nk; ++t)
+        ptx::mbar_wait(kfull(t % KS), (t / KS) & 1, &never, kDrainLimitNs);
+      for (int t = max(0, nv - VS); t < nv; ++t)
+        ptx::mbar_wait(vfull(t % VS), (t / VS) & 1, &never, kDrainLimitNs);
+      for (int c = max(0, nr - RS); c < nr; ++c)
+        ptx::mbar_wait(rfull(c % RS), (c / RS) & 1, &never, kDrainLimitNs);
+    }
     if (bad_cta) atomicOr(p.status, kStatusBadSeq);
   }
   if (aborted_cta || bad_cta)
@@ -633,6 +644,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);
   }
+  finish_split<G>(p, b, h, first_token_row(p, b));
 }
 
 }  // namespace relattn

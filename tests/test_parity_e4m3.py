@@ -202,7 +202,7 @@ def test_previous_model_full_layer(ra, name):
 
 
 def test_injected_wait_limit_times_out_cleanly(ra):
-    """As for the bf16 kernel: a 1 us wait bound makes the E4M3 kernel abort
+    """As for the bf16 kernel: a 1 ns wait bound makes the E4M3 kernel abort
     promptly with TIMEOUT and NaN rows; the default bound then works again."""
     import time
     case = W.make_workload("full_100k", seed=4, device="cuda", num_q_heads=12, num_kv_heads=2)
@@ -218,7 +218,7 @@ def test_injected_wait_limit_times_out_cleanly(ra):
     torch.cuda.synchronize()
     assert ws.read_status() == ra.REL_ATTN_OK
     try:
-        ra.rel_attn_set_wait_limit(1000)
+        ra.rel_attn_set_wait_limit(1)
         t0 = time.perf_counter()
         out, lse = call()
         torch.cuda.synchronize()
