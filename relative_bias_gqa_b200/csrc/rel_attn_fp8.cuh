@@ -33,7 +33,7 @@ struct Fp8Config {
   static constexpr int NG = 2, RG = G;
   static_assert(2 * G <= N && 3 * G <= NP && G % 2 == 0, "group size");
   static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
-  static constexpr int kKSlots = 3, kVSlots = 5, kRSlots = 2;
+  static constexpr int kKSlots = 4, kVSlots = 6, kRSlots = 1;
   static constexpr int kTile8 = 128 * 128;                      // 128 keys x 128 B
   static constexpr int kPage8 = 64 * 128;
   static constexpr int kRHalf = 128 * 128;                      // 128 rows x 64 dims bf16
