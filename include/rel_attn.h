@@ -80,11 +80,8 @@ typedef struct rel_attn_shape {
 } rel_attn_shape;
 
 /*
- * rel_attn_decode -- the whole hot path in one kernel launch: the split-KV
- * partial kernel, whose CTAs count their finished splits per (sequence, KV
- * head) in the workspace; the last CTA of each merges the splits' partials
- * (the LSE merge).  Batches with more than 960 (sequence, KV head) pairs
- * merge with a second kernel instead.
+ * rel_attn_decode -- the whole hot path: split-KV partial kernel, then (when
+ * num_splits > 1) the LSE-merge combine kernel.
  *
  *   q           bf16 [B, T, Hq, D], row-major.
  *   k_cache     bf16 [num_pages, Hkv, P, D]: one (page, KV head) is a
@@ -102,9 +99,7 @@ typedef struct rel_attn_shape {
  *   lse         fp32 [B, T, Hq] natural-log LSE of the scaled logits, or NULL.
  *   workspace   device scratch of at least rel_attn_workspace_bytes(shape,
  *               num_splits) bytes, 256-byte aligned, prepared once with
- *               rel_attn_workspace_init (it holds the device status word,
- *               the merge counters -- every call leaves them at zero again
- *               -- and the per-split partials).
+ *               rel_attn_workspace_init (it holds the device status word).
  *
  * Device-side problems (seq_len out of range, a block-table entry outside
  * the pool, a wait that exceeded its bound) do not fault: they set bits in
@@ -130,10 +125,9 @@ int rel_attn_decode(const rel_attn_shape* shape, const void* q,
  * rel_attn_choose_splits).  With num_splits == 1 the partial call writes
  * out/lse itself and the combine call is a no-op.  With num_splits > 1 the
  * partial call writes the per-split (normalised output, lse) pairs into the
- * workspace -- fp32 [S][B*T*Hq] lse from byte 4096 (after the status word
- * and rel_attn_decode's merge counters), then fp32 [S][B*T*Hq][D] outputs at
- * the next 256-byte boundary; a split with no visible key holds lse = -inf
- * and zeros -- and the combine call merges them:
+ * workspace -- fp32 [S][B*T*Hq] lse after the 256-byte header, then fp32
+ * [S][B*T*Hq][D] outputs at the next 256-byte boundary; a split with no
+ * visible key holds lse = -inf and zeros -- and the combine call merges them:
  *   lse = ln sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) o_s.
  */
 int rel_attn_partial(const rel_attn_shape* shape, const void* q,
@@ -295,8 +289,8 @@ int rel_attn_kv_write(const rel_attn_shape* shape, const void* k_new, const void
  * (num_splits <= 0: the heuristic's choice).  0 when the shape is invalid. */
 size_t rel_attn_workspace_bytes(const rel_attn_shape* shape, int num_splits);
 
-/* Zero the workspace status word and merge counters (asynchronous on
- * `stream`).  Call once after allocating a workspace. */
+/* Zero the workspace status word (asynchronous on `stream`).  Call once
+ * after allocating a workspace and after reading a non-zero status. */
 int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bound, in nanoseconds, of each device-side wait in launches made after

@@ -220,18 +220,11 @@ int splits_heuristic(const rel_attn_shape* s, int window, int sm_count) {
   return (int)S;
 }
 
-// Status word (kHeaderBytes), then for S > 1 the fused-merge counters and the
-// per-split partials (lse from kPartialsOffset, outputs after them).
 size_t workspace_for(const rel_attn_shape* s, int S) {
   if (S <= 1) return kHeaderBytes;
   const size_t rows = (size_t)s->batch * s->q_tokens * s->num_q_heads;
-  return kPartialsOffset + align256((size_t)S * rows * sizeof(float)) +
+  return kHeaderBytes + align256((size_t)S * rows * sizeof(float)) +
          (size_t)S * rows * kHeadDim * sizeof(float);
-}
-
-// The fused merge needs a counter per (sequence, KV head).
-bool fused_merge_fits(const rel_attn_shape* s) {
-  return (long long)s->batch * s->num_kv_heads <= kMaxFusedUnits;
 }
 
 int probe_device(int* dev_out) {
@@ -422,9 +415,7 @@ int rel_attn_set_wait_limit(unsigned long long limit_ns) {
 
 int rel_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < kHeaderBytes) return REL_ATTN_ERR_INVALID_ARG;
-  // the status word and, when the workspace has them, the merge counters
-  const size_t n = workspace_bytes < (size_t)kPartialsOffset ? kHeaderBytes : (size_t)kPartialsOffset;
-  return cudaMemsetAsync(workspace, 0, n, (cudaStream_t)stream) == cudaSuccess
+  return cudaMemsetAsync(workspace, 0, kHeaderBytes, (cudaStream_t)stream) == cudaSuccess
              ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
 }
 
@@ -492,9 +483,8 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->lse = lse;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   prm->status = reinterpret_cast<unsigned*>(ws);
-  prm->ws_lse = reinterpret_cast<float*>(ws + kPartialsOffset);
-  prm->ws_o = reinterpret_cast<float*>(ws + kPartialsOffset + align256((size_t)S * rows * sizeof(float)));
-  prm->counters = nullptr;                   // set by the entry points that merge in the kernel
+  prm->ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes);
+  prm->ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
   const unsigned long long wl = g_wait_limit_ns.load(std::memory_order_relaxed);
   prm->timeout_ns = wl ? wl : kDefaultTimeoutNs;
   prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
@@ -558,8 +548,8 @@ int launch_combine(const rel_attn_shape* shape, int S, void* out, float* lse, vo
                    cudaStream_t st) {
   const size_t rows = (size_t)shape->batch * shape->q_tokens * shape->num_q_heads;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  const float* ws_lse = reinterpret_cast<const float*>(ws + kPartialsOffset);
-  const float* ws_o = reinterpret_cast<const float*>(ws + kPartialsOffset + align256((size_t)S * rows * sizeof(float)));
+  const float* ws_lse = reinterpret_cast<const float*>(ws + kHeaderBytes);
+  const float* ws_o = reinterpret_cast<const float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)rows);
@@ -592,10 +582,8 @@ int rel_attn_decode(const rel_attn_shape* shape, const void* q, const void* k_ca
                    out, lse, workspace, workspace_bytes, &prm, &S, &di);
   if (rc != REL_ATTN_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool fused = S > 1 && fused_merge_fits(shape);
-  if (fused) prm.counters = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(workspace) + kCounterOffset);
   rc = launch_partial_any(prm, shape, S, st, *di);
-  if (rc != REL_ATTN_OK || S == 1 || fused) return rc;
+  if (rc != REL_ATTN_OK || S == 1) return rc;
   return launch_combine(shape, S, out, lse, workspace, st);
 }
 
@@ -625,10 +613,8 @@ int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q, const void*
                    out, lse, workspace, workspace_bytes, &prm, &S, &di, k_scale, v_scale, true);
   if (rc != REL_ATTN_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool fused = S > 1 && fused_merge_fits(shape);
-  if (fused) prm.counters = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(workspace) + kCounterOffset);
   rc = launch_partial_e4m3(prm, shape, S, st, *di);
-  if (rc != REL_ATTN_OK || S == 1 || fused) return rc;
+  if (rc != REL_ATTN_OK || S == 1) return rc;
   return launch_combine(shape, S, out, lse, workspace, st);
 }
 
@@ -716,8 +702,8 @@ extern "C" int rel_attn_prefill(const rel_attn_shape* shape, const void* q, cons
   const size_t rows = (size_t)shape->batch * C * shape->num_q_heads;
   if (workspace_bytes < workspace_for(shape, S)) return REL_ATTN_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  prm.ws_lse = reinterpret_cast<float*>(ws + kPartialsOffset);
-  prm.ws_o = reinterpret_cast<float*>(ws + kPartialsOffset + align256((size_t)S * rows * sizeof(float)));
+  prm.ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes);
+  prm.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + align256((size_t)S * rows * sizeof(float)));
   prm.rows_total = (int)rows;
   prm.seq_stride = C;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -884,10 +870,8 @@ extern "C" int rel_attn_decode_static(const rel_attn_shape* shape, const void* q
   if (rc != REL_ATTN_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left there: the status word
-  // and the merge counters must start at zero (every launch leaves its
-  // counters at zero again, but a call may follow one that did not finish);
-  // the per-split partials are rewritten in full.
-  if (cudaMemsetAsync(scratch, 0, S > 1 ? (size_t)kPartialsOffset : kHeaderBytes, st) != cudaSuccess) {
+  // must start at zero; the per-split partials are rewritten in full.
+  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, st) != cudaSuccess) {
     cudaGetLastError();
     return REL_ATTN_ERR_CUDA;
   }

@@ -295,13 +295,12 @@ def rel_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, rel_table, wind
 def prefill_workspace_bytes(shape: RelAttnShape, num_splits: int) -> int:
     """Workspace bytes rel_attn_prefill needs: the status word, plus, with
     more than one split, every row's partials (the layout of the decode
-    workspace for B * C rows: partials from byte 4096).  num_splits <= 0
-    assumes up to 256."""
+    workspace for B * C rows).  num_splits <= 0 assumes up to 256."""
     S = num_splits if num_splits > 0 else 256
     rows = shape.batch * shape.q_tokens * shape.num_q_heads
     if S == 1:
         return 256
-    return 4096 + (S * rows * 4 + 255) // 256 * 256 + S * rows * 128 * 4
+    return 256 + (S * rows * 4 + 255) // 256 * 256 + S * rows * 128 * 4
 
 
 def rel_attn_kv_write(k_new, v_new, conv_w, k_raw, v_raw, k_cache, v_cache, block_table,

@@ -129,9 +129,7 @@ GOOD = [dict(num_q_heads=48, num_kv_heads=8, q_tokens=t) for t in range(1, 10)] 
 def test_supported_group_shapes(ra, kw):
     s = shape(ra, **kw)
     rows = kw["q_tokens"] * kw["num_q_heads"]
-    # status word and merge counters (4 KB), then lse and output partials
-    assert ra.rel_attn_workspace_bytes(s, 3) == 4096 + (3 * rows * 4 + 255) // 256 * 256 + 3 * rows * 128 * 4
-    assert ra.rel_attn_workspace_bytes(s, 1) == 256
+    assert ra.rel_attn_workspace_bytes(s, 3) == 256 + (3 * rows * 4 + 255) // 256 * 256 + 3 * rows * 128 * 4
 
 
 def test_e4m3_only_for_one_token(ra):
@@ -179,8 +177,7 @@ def test_workspace_bytes(ra):
     s = shape(ra)
     assert ra.rel_attn_workspace_bytes(s, 1) == 256
     rows = 48
-    # status word + merge counters (4 KB), lse partials, output partials
-    want = 4096 + ((18 * rows * 4 + 255) // 256) * 256 + 18 * rows * 128 * 4
+    want = 256 + ((18 * rows * 4 + 255) // 256) * 256 + 18 * rows * 128 * 4
     assert ra.rel_attn_workspace_bytes(s, 18) == want
     assert ra.rel_attn_workspace_bytes(s, 256) > ra.rel_attn_workspace_bytes(s, 18)
 
