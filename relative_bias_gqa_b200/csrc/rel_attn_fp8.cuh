@@ -106,7 +106,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   if (g.L < T || g.L > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
     fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-    finish_split<G>(p, b, h, first_token_row(p, b));
     return;
   }
   g.p0 = g.L - T;
@@ -116,7 +115,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {
     fill_rows<G>(p, first_token_row(p, b), h, s_idx, 0.f, -INFINITY);
-    finish_split<G>(p, b, h, first_token_row(p, b));
     return;
   }
 
@@ -644,7 +642,6 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);
   }
-  finish_split<G>(p, b, h, first_token_row(p, b));
 }
 
 }  // namespace relattn

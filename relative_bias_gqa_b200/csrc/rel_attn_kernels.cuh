@@ -102,10 +102,6 @@ struct alignas(64) DecodeParams {
   // one sequence, each attending causally to everything before it.
   int cps, seq_stride, tok_off, len_off;
   int rows_total;       // rows of the partial buffers: all query tokens x Hq
-  // Fused merge: one counter per (grid z-index, KV head); the CTA that
-  // finishes last merges the splits' partials itself.  Null: the partials
-  // are left for the combine kernel.
-  unsigned* counters;
   int ex;               // distances d < ex are their own bucket
   int nl;               // tail buckets: bucket = ex + max{k < nl : edges[k] <= d}
   float scale_log2;     // log2(e) / sqrt(D)
@@ -410,85 +406,6 @@ __device__ void fill_rows(const DecodeParams& p, int tok0, int h, int s, float o
   }
 }
 
-// Workspace layout (bytes): the status word at 0; the fused-merge counters
-// from kCounterOffset; the per-split partials from kPartialsOffset (lse,
-// then outputs).  Launches with more units than the counters hold use the
-// combine kernel instead.
-constexpr int kCounterOffset = 256;
-constexpr int kPartialsOffset = 4096;
-constexpr int kMaxFusedUnits = (kPartialsOffset - kCounterOffset) / 4;
-
-// LSE merge of the S splits' partials of one (sequence, KV head): rows
-// row0..row0+T-1 (tokens) x the group's G heads; thread (row, 4 head dims).
-// lse = max + ln sum_s exp(lse_s - max), out = sum_s w_s o_s / sum_s w_s;
-// splits with lse_s = -inf are skipped, a NaN partial makes the row NaN.
-template <int G>
-__device__ void merge_rows(const DecodeParams& p, int row0, int h) {
-  const int S = p.num_splits, rows = p.rows_total;
-  for (int e = threadIdx.x; e < p.T * G * 32; e += blockDim.x) {
-    const int n = e >> 5, q = e & 31;
-    const int t = n / G, gg = n - t * G;
-    const int row = (row0 + t) * p.Hq + h * G + gg;
-    float mx = -INFINITY;
-    bool nan = false;
-#pragma unroll 8
-    for (int s = 0; s < S; ++s) {
-      const float l = __ldcg(p.ws_lse + (size_t)s * rows + row);
-      nan |= (l != l);
-      mx = fmaxf(mx, l);
-    }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float sum = 0.f;
-    if (!nan && mx != -INFINITY) {
-#pragma unroll 8
-      for (int s = 0; s < S; ++s) {
-        const float l = __ldcg(p.ws_lse + (size_t)s * rows + row);
-        const float w = (l == -INFINITY) ? 0.f : expf(l - mx);
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(p.ws_o + ((size_t)s * rows + row) * kHeadDim) + q);
-        sum += w;
-        acc.x = fmaf(w, o.x, acc.x);
-        acc.y = fmaf(w, o.y, acc.y);
-        acc.z = fmaf(w, o.z, acc.z);
-        acc.w = fmaf(w, o.w, acc.w);
-      }
-    }
-    const float qnan = __int_as_float(0x7fc00000);
-    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
-    float4 r = nan ? make_float4(qnan, qnan, qnan, qnan)
-                   : make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (p.out_fp32) {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * kHeadDim)[q] = r;
-    } else {
-      const __nv_bfloat162 lo2 = __floats2bfloat162_rn(r.x, r.y), hi2 = __floats2bfloat162_rn(r.z, r.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
-      pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
-      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * kHeadDim)[q] = pk;
-    }
-    if (p.lse && q == 0) p.lse[row] = nan ? qnan : (sum > 0.f ? mx + logf(sum) : -INFINITY);
-  }
-}
-
-// Called once by every CTA of a launch, after its last write: the CTA whose
-// arrival completes its (sequence, KV head)'s count merges the splits and
-// resets the counter for the next launch.  No CTA waits for another.
-template <int G>
-__device__ void finish_split(const DecodeParams& p, int b, int h, int row0) {
-  if (p.counters == nullptr || p.num_splits <= 1) return;
-  __shared__ int s_last;
-  __threadfence();                           // this CTA's partials, device-wide
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(p.counters + (size_t)b * p.Hkv + h, 1u);
-    s_last = (prev == (unsigned)p.num_splits - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();                           // every split's partials are visible
-  merge_rows<G>(p, row0, h);
-  if (threadIdx.x == 0) p.counters[(size_t)b * p.Hkv + h] = 0u;
-}
-
 // T (query tokens) is a template parameter: every per-row loop below runs
 // over the NQ = T*G live rows only, fully unrolled.
 template <int N, int G, int NG, int T>
@@ -533,7 +450,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   if (L_seq < p.seq_stride || L_seq > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
     fill_rows<G>(p, row0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-    finish_split<G>(p, b, h, row0);
     return;
   }
   g.p0 = g.L - T;
@@ -543,7 +459,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {                       // a trailing split with no page
     fill_rows<G>(p, row0, h, s_idx, 0.f, -INFINITY);
-    finish_split<G>(p, b, h, row0);
     return;
   }
 
@@ -1228,7 +1143,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, KC::kTmemCols);
   }
-  finish_split<G>(p, b, h, row0);
 }
 
 // LSE merge of per-split partial results: one CTA per (b, t, hq) row; its
