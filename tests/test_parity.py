@@ -370,6 +370,55 @@ def test_verify_256k_every_token_count(ra, T):
         check(*run_gpu(ra, case, splits), *ref)
 
 
+# ------------------------------------------------------- merge entry points
+def test_split_phase_partial_then_combine(ra):
+    """rel_attn_partial + rel_attn_combine (the split-phase entry points)
+    give exactly what rel_attn_decode gives, and match the oracle."""
+    case = small(0, T=3, Hkv=2, lens=[5000, 700, 129])
+    ref = run_oracle(case)
+    for splits in (2, 7, 40):
+        prep = ra.Prepared(case.q, case.k_cache, case.v_cache, case.block_table, case.seq_lens,
+                           case.rel_table, case.window, splits, max_seq_len=case.max_seq_len,
+                           out_fp32=True)
+        prep.partial()
+        prep.combine()
+        torch.cuda.synchronize()
+        a = (prep.out.clone(), prep.lse.clone())
+        check(*a, *ref)
+        prep.decode()
+        torch.cuda.synchronize()
+        assert torch.equal(prep.out, a[0]) and torch.equal(prep.lse, a[1])
+        assert prep.workspace.read_status() == ra.REL_ATTN_OK
+
+
+def test_many_sequences_and_heads(ra):
+    """968 (sequence, KV head) pairs in one call: 121 sequences x 8 KV heads,
+    lengths 2..901, checked on four sequences."""
+    lens = [(37 * i) % 900 + 2 for i in range(121)]
+    case = W.make_case(seq_lens=lens, q_tokens=1, num_q_heads=48, num_kv_heads=8, window=0,
+                       num_buckets=1280, seed=12).to("cuda")
+    idx = [0, 1, 60, 120]
+    ref_o, ref_l = run_oracle(case, batch_indices=idx)
+    for splits in (3, 0):
+        out, lse = run_gpu(ra, case, splits)
+        check(out[idx], lse[idx], ref_o[idx], ref_l[idx])
+
+
+def test_one_workspace_across_shapes(ra):
+    """One workspace serves calls of different shapes and split counts in
+    turn (it holds only the status word and each call's own partials)."""
+    from relative_bias_gqa_b200.rel_attn import Workspace
+    big = small(0, T=2, Hkv=3, lens=[3000, 100, 2500])
+    shape = ra.shape_of(big.q, big.k_cache, big.block_table, big.rel_table, out_fp32=True)
+    ws = Workspace.for_shape(shape, 64, "cuda")
+    cases = [big, small(2000, T=1, Hkv=2), small(0, T=5, Hkv=1, lens=[900, 4000])]
+    refs = [run_oracle(c) for c in cases]
+    for _ in range(2):
+        for c, ref, splits in zip(cases, refs, (64, 5, 17)):
+            check(*run_gpu(ra, c, splits, workspace=ws), *ref)
+    assert ws.read_status() == ra.REL_ATTN_OK
+
+
 # ------------------------------------------------------------- error paths
 def test_bad_sequence_length_reports_and_writes_nan(ra):
     case = small(500, T=1)
