@@ -16,9 +16,12 @@
 //   O^T = V8^T . [P_hi; P_mid; P_lo]^T   P = P_hi + P_mid / 16 + P_lo / 256,
 //                                   12 significant bits
 //   X^T = R_chunk . Q^T             bf16 (kind::f16) as in the bf16 kernel
-// Roles as in the bf16 one-token kernel: warp 0 TMA producer (K8 and V8
-// page tiles, 8 KB per page, and relative-row chunks, each in its own
-// ring), warp 1 MMA issuer, two softmax groups of 4 warps alternating tiles.
+// Roles: warp 0 TMA producer (K8 and V8 page tiles, 8 KB per page, and
+// relative-row chunks, each in its own ring), warp 1 issues S and X, warp 10
+// issues P.V, two softmax groups of 4 warps (2..9) alternate tiles.  The two
+// MMA issuers run side by side: a single issuing thread spends about a
+// microsecond per tile on its waits, descriptors and eight MMA issues, more
+// than the tile's bytes take to arrive at the HBM rate.
 // The K scale and the query's per-row power of two fold into the logit
 // scale, the V scale into the output.  The lazy reference max keeps
 // P <= 2^8 here, inside E4M3 range.
@@ -32,7 +35,8 @@ struct Fp8Config {
   static constexpr int NP = 32;                                 // P.V columns: 3 terms x G rows
   static constexpr int NG = 2, RG = G;
   static_assert(2 * G <= N && 3 * G <= NP && G % 2 == 0, "group size");
-  static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
+  static constexpr int kPvWarp = 2 + 4 * NG;                   // after the softmax warps
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + 32;
   static constexpr int kKSlots = 4, kVSlots = 6, kRSlots = 1;
   static constexpr int kTile8 = 128 * 128;                      // 128 keys x 128 B
   static constexpr int kPage8 = 64 * 128;
@@ -54,11 +58,14 @@ struct Fp8Config {
   static constexpr int oEdges = oQf + 64;
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
   // kfull/kempty[KS] vfull/vempty[VS] rfull/rempty[RS] s_full/s_empty[2]
-  // p_full[2] o_full/o_empty[2] x_full/x_empty[2] drain
-  static constexpr int kNumBars = 2 * (kKSlots + kVSlots + kRSlots) + 4 + 2 + 4 + 4 + 1;
+  // p_full[2] o_full/o_empty[2] x_full/x_empty[2] drain (S issuer) drain (P.V issuer)
+  static constexpr int kNumBars = 2 * (kKSlots + kVSlots + kRSlots) + 4 + 2 + 4 + 4 + 2;
   // tmem base, abort flag, bad-page flag, K / V tiles and relative chunks issued
   static constexpr int oMisc = oBar + kNumBars * 8;
-  static constexpr int kBytes = oMisc + 32;
+  // per K slot: 1 if its tile starts a new relative-row chunk (producer ->
+  // S issuer, published by the slot's full barrier)
+  static constexpr int oChunkFlag = oMisc + 32;
+  static constexpr int kBytes = oChunkFlag + align_up(kKSlots, 16);
   static constexpr int kAllocBytes = kBytes + 1024;
   static constexpr int kTmemCols = 128;                         // S[2] 32 + O[2] 64 + X[2] 32
   static_assert(kAllocBytes <= 232448, "shared memory budget exceeded");
@@ -137,6 +144,8 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t x_full = bar0 + 8u * (kB + 10);    // +8*group
   const uint32_t x_empty = bar0 + 8u * (kB + 12);
   const uint32_t drain_bar = bar0 + 8u * (kB + 14);
+  const uint32_t drain_pv = bar0 + 8u * (kB + 15);
+  uint8_t* chunk_flag = smem + FC::oChunkFlag;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + FC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 4);
   volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + FC::oMisc + 8);
@@ -161,6 +170,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       ptx::mbar_init(x_empty + 8u * i, kSoftmaxThreads);
     }
     ptx::mbar_init(drain_bar, 1);
+    ptx::mbar_init(drain_pv, 1);
     *abort_flag = 0;
     *bad_page_flag = 0;
     issued[0] = issued[1] = issued[2] = 0;
@@ -175,7 +185,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     if (warp == 1) {
       ptx::tmem_alloc(ptx::smem_addr(tmem_holder), FC::kTmemCols);
       ptx::tmem_relinquish();
-    } else {
+    } else if (warp != FC::kPvWarp) {
       const int st = tid - 64;                  // softmax thread 0..255
       const int sw = st >> 5;                   // its warp 0..7
       // bf16 Q for X: rows 0..G-1 the group's heads, other rows zero,
@@ -278,6 +288,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(kempty(ti % KS), ((ti / KS) & 1) ^ 1, abort_flag, tlim));
       if (!ok) break;
       if (lane == 0) {
+        chunk_flag[ti % KS] = tp.chunk ? 1 : 0;
         ptx::mbar_arrive_expect_tx(kfull(ti % KS), tp.npg * FC::kPage8);
         ptx::tma_load_2d(kslot(ti), &p.tmap_k, kfull(ti % KS), 0, row0, pol);
         if (tp.npg > 1) ptx::tma_load_2d(kslot(ti) + FC::kPage8, &p.tmap_k, kfull(ti % KS), 0, row1, pol);
@@ -299,52 +310,25 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       issued[2] = nr;
     }
   }
-  // ------------------------------------------------------------ MMA issuer
+  // ------------------------------------------------------- S and X issuer
   else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdescS = ptx::idesc_e4m3(128, N, false, false);    // K8 . [Q_hi; Q_lo]
-      constexpr uint32_t kIdescPV = ptx::idesc_e4m3(128, NP, true, true);    // V8^T . [P terms]
       constexpr uint32_t kIdescX = ptx::idesc_bf16(128, N, false, false);    // R . Q
       const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + FC::oK, 16, 1024);    // K8, K-major
       const uint64_t q8desc = ptx::sdesc_sw128(sbase + FC::oQ8, 16, 1024);   // Q8, K-major
-      const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + FC::oV, 16, 1024);    // V8^T, MN-major
-      const uint64_t pdesc0 = ptx::sdesc_noswz(sbase + FC::oP, 256, 128);    // P terms, MN-major
       const uint64_t rdesc0 = ptx::sdesc_sw128(sbase + FC::oR, 16, 1024);    // R chunk, K-major
       const uint64_t qdesc = ptx::sdesc_sw128(sbase + FC::oQ, 16, 1024);     // bf16 Q, K-major
-      int i = 0, nr = 0;                       // tiles, chunks issued
+      int nr = 0;                              // chunks issued
       int cg[2] = {0, 0};                      // chunks per group
-      PlanState ps0(p.nl), ps1(p.nl);
-      bool ok = true;
-      auto issue_pv = [&](int j) -> bool {
-        if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
-        if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
-        if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
-        ptx::tc_fence_after();
-        const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * FC::kTile8) >> 4);
-        const uint64_t pb = pdesc0 + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
-        // K = 32 keys per MMA: 32 rows of the V tile (4 KB), four 8-key
-        // core-matrix groups of P (1 KB)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::umma_e4m3(tO + (j & 1) * NP, va + (uint64_t)((kk * 4096) >> 4),
-                         pb + (uint64_t)((kk * 1024) >> 4), kIdescPV, kk > 0);
-        ptx::umma_commit(o_full + 8u * (j & 1));
-        ptx::umma_commit(vempty(j % VS));
-        return true;
-      };
       for (int ti = 0; ti < g.ntiles; ++ti) {
         const int gq = ti & 1;
-        const TilePlan tp = plan_tile<128>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
-        bool pv_pending = i > 0;
-        if (pv_pending && !ptx::mbar_try_wait(kfull(ti % KS), (ti / KS) & 1)) {
-          if (!(ok = issue_pv(i - 1))) break;
-          pv_pending = false;
-        }
-        if (tp.chunk) {
+        if (!ptx::mbar_wait(kfull(ti % KS), (ti / KS) & 1, abort_flag, tlim)) break;
+        if (chunk_flag[ti % KS]) {
           const int c = cg[gq];
-          ok = ptx::mbar_wait(rfull(nr % RS), (nr / RS) & 1, abort_flag, tlim) &&
-               ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
-          if (!ok) break;
+          if (!ptx::mbar_wait(rfull(nr % RS), (nr / RS) & 1, abort_flag, tlim) ||
+              !ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim))
+            break;
           ptx::tc_fence_after();
           const uint64_t rd = rdesc0 + (uint64_t)(((nr % RS) * FC::kRBytes) >> 4);
 #pragma unroll
@@ -358,27 +342,49 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
           ++nr;
           cg[gq] = c + 1;
         }
-        ok = ptx::mbar_wait(kfull(ti % KS), (ti / KS) & 1, abort_flag, tlim) &&
-             ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
-        if (!ok) break;
+        if (!ptx::mbar_wait(s_empty + 8u * gq, ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
         ptx::tc_fence_after();
-        {
-          const uint64_t kd = kdesc0 + (uint64_t)(((ti % KS) * FC::kTile8) >> 4);
-          // K = 32 dims (32 B of each 128 B row) per MMA
+        const uint64_t kd = kdesc0 + (uint64_t)(((ti % KS) * FC::kTile8) >> 4);
+        // K = 32 dims (32 B of each 128 B row) per MMA
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_e4m3(tS + (i & 1) * N, kd + (uint64_t)((kk * 32) >> 4),
-                           q8desc + (uint64_t)((kk * 32) >> 4), kIdescS, kk > 0);
-          ptx::umma_commit(s_full + 8u * (i & 1));
-          ptx::umma_commit(kempty(ti % KS));
-        }
-        if (pv_pending && !(ok = issue_pv(i - 1))) break;
-        ++i;
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_e4m3(tS + gq * N, kd + (uint64_t)((kk * 32) >> 4),
+                         q8desc + (uint64_t)((kk * 32) >> 4), kIdescS, kk > 0);
+        ptx::umma_commit(s_full + 8u * gq);
+        ptx::umma_commit(kempty(ti % KS));
       }
-      if (ok && i > 0) ok = issue_pv(i - 1);
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
       ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
+    }
+    __syncwarp();
+  }
+  // ----------------------------------------------------------- P.V issuer
+  else if (warp == FC::kPvWarp) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = ptx::idesc_e4m3(128, NP, true, true);    // V8^T . [P terms]
+      const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + FC::oV, 16, 1024);    // V8^T, MN-major
+      const uint64_t pdesc0 = ptx::sdesc_noswz(sbase + FC::oP, 256, 128);    // P terms, MN-major
+      for (int j = 0; j < g.ntiles; ++j) {
+        if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim) ||
+            !ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim) ||
+            !ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim))
+          break;
+        ptx::tc_fence_after();
+        const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * FC::kTile8) >> 4);
+        const uint64_t pb = pdesc0 + (uint64_t)(((j & 1) * FC::kPBufBytes) >> 4);
+        // K = 32 keys per MMA: 32 rows of the V tile (4 KB), four 8-key
+        // core-matrix groups of P (1 KB)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_e4m3(tO + (j & 1) * NP, va + (uint64_t)((kk * 4096) >> 4),
+                         pb + (uint64_t)((kk * 1024) >> 4), kIdescPV, kk > 0);
+        ptx::umma_commit(o_full + 8u * (j & 1));
+        ptx::umma_commit(vempty(j % VS));
+      }
+      ptx::umma_commit(drain_pv);
+      volatile int never = 0;
+      ptx::mbar_wait(drain_pv, 0, &never, kDrainLimitNs);
     }
     __syncwarp();
   }
