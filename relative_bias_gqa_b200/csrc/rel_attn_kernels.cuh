@@ -4,7 +4,9 @@
 //   warp 0      TMA producer: walks the split's pages through the block table
 //               and streams K/V page tiles (and relative-table row chunks)
 //               into a ring of 64 KB shared-memory stages.
-//   warp 1      MMA issuer (one thread): tcgen05.mma with fp32 accumulators
+//   warp 1      MMA issuer (one thread; in most instances it issues S and X
+//               and a warp after the softmax warps issues P.V): tcgen05.mma
+//               with fp32 accumulators
 //               in tensor memory, "swap-AB" orientation so that keys (and
 //               head-dim for P.V) fill the 128-row M side and the GQA
 //               group's G heads x T tokens are the N side:
@@ -125,7 +127,15 @@ struct KernelConfig {
   // rows.  N = 32 / 48 / 64 (2..9 tokens): every group takes every tile, each
   // with its own block of rows (a column split of S^T, X^T and O^T).
   static constexpr bool kAlt = (N == 16);
-  static constexpr int kThreads = 64 + kSoftmaxThreads * NG;
+  // warp 0 producer, warp 1 MMA issuer, the softmax warps.  kSplitIssue:
+  // warp 1 issues S and X only and a warp after the softmax warps issues
+  // P.V.  Measured on B200 (256K-key verify step, tokens 1..9): faster with
+  // two groups and with an odd token count over four groups (7 and 9 tokens
+  // at G = 6: 274 -> 267 and 543 -> 510 us), slower with an even one (6 and 8
+  // tokens: 262 -> 271 and 251 -> 260 us).
+  static constexpr bool kSplitIssue = (NG == 2) || (T % 2 == 1);
+  static constexpr int kPvWarp = kSplitIssue ? 2 + 4 * NG : -1;
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + (kSplitIssue ? 32 : 0);
   static constexpr int kConsumers = kAlt ? kSoftmaxThreads : kSoftmaxThreads * NG;  // arrivals per tile
   static constexpr int kXTables = kAlt ? NG : 1;               // relative chunks in flight (X, Y)
   // row capacity of a group: N / NG, or more when the tokens do not split
@@ -162,11 +172,14 @@ struct KernelConfig {
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
   // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s_full[2],
   //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[kXTables],
-  //           x_empty[kXTables], drain
-  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 11 + 2 * kXTables;
+  //           x_empty[kXTables], drain (S issuer), drain (P.V issuer)
+  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 12 + 2 * kXTables;
   // tmem base, abort flag, bad-page flag, K-ring and V-ring items issued
   static constexpr int oMisc = oBar + kNumBars * 8;
-  static constexpr int kBytes = oMisc + 32;
+  // per K slot: 1 if its item is a relative-row chunk, 0 a K tile (producer
+  // -> S issuer, published by the slot's full barrier)
+  static constexpr int oItemFlag = oMisc + 32;
+  static constexpr int kBytes = oItemFlag + align_up(kKSlots, 16);
   static constexpr int kAllocBytes = kBytes + 1024;            // 1024-byte alignment slack
   // TMEM columns: S[2] (N each), O[2] (2N each: the P_hi and P_lo halves),
   // per group X0 (and X1 for 136-row chunks)
@@ -485,6 +498,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t x_full = bar0 + 8u * (kB + 10);   // +8*group
   const uint32_t x_empty = bar0 + 8u * (kB + 10 + KC::kXTables);
   const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * KC::kXTables);
+  const uint32_t drain_pv = drain_bar + 8u;
+  uint8_t* item_flag = smem + KC::oItemFlag;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 4);
   volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 8);
@@ -517,6 +532,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       ptx::mbar_init(x_empty + 8u * gq, KC::kConsumers);
     }
     ptx::mbar_init(drain_bar, 1);
+    ptx::mbar_init(drain_pv, 1);
     *abort_flag = 0;
     *bad_page_flag = 0;
     issued[0] = issued[1] = 0;
@@ -531,7 +547,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     if (warp == 1) {
       ptx::tmem_alloc(ptx::smem_addr(tmem_holder), KC::kTmemCols);
       ptx::tmem_relinquish();
-    } else {
+    } else if (!KC::kSplitIssue || warp != KC::kPvWarp) {
       const int st = tid - 64;
       const int nst = kSoftmaxThreads * NG;
       // Q group tile, 128B-swizzled K-major: query slot n holds (token t,
@@ -602,6 +618,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           if (!ok) break;
           if (lane == 0) {
             const uint32_t st = kslot(k);
+            item_flag[k % KS] = 1;
             ptx::mbar_arrive_expect_tx(kfull(k % KS), 2 * KC::kRHalfBytes);
             ptx::tma_load_3d(st, &p.tmap_r, kfull(k % KS), 0, c0, h);
             ptx::tma_load_3d(st + KC::kRHalfBytes, &p.tmap_r, kfull(k % KS), 64, c0, h);
@@ -622,6 +639,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (lane == 0) {
           const uint32_t st = kslot(k);
           const uint32_t fb = kfull(k % KS);
+          item_flag[k % KS] = 0;
           ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
           for (int pi = 0; pi < tp.npg; ++pi) {
             const int row = pi ? rows1[ti & 1] : rows0[ti & 1];
@@ -656,25 +674,162 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       issued[1] = i_v;
     }
   }
-  // ------------------------------------------------------------ MMA issuer
+  // ------------------------------------------------------- S and X issuer
+  // With kSplitIssue, S / X and P.V are issued by two warps side by side: one
+  // issuing thread spends most of a microsecond per tile on its waits,
+  // descriptors and MMA issues, close to what the tile's bytes take at the
+  // HBM rate.  Otherwise this thread issues both, P.V of the previous tile
+  // first unless this tile's K data has already landed.
   else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
+      if constexpr (KC::kSplitIssue) {
+        constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
+        // Base descriptors; every MMA operand below is one of these plus a
+        // constant byte offset (the address field is the low 14 bits, >> 4).
+        const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
+        const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
+        int k = 0;                               // K-ring items taken
+        int cg[2] = {0, 0};                      // chunks issued per group
+        for (int ti = 0; ti < g.ntiles; ++ti) {
+          const int gq = KC::kAlt ? (ti & 1) : 0;
+          if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
+          if (item_flag[k % KS]) {
+            // the tile's new relative-row chunk came first: X = R_chunk . Q
+            const int c = cg[gq];
+            if (!ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim)) break;
+            ptx::tc_fence_after();
+            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
+              const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+              ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
+              if constexpr (ROWS > 128)
+                ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
+            }
+            ptx::umma_commit(x_full + 8u * gq);
+            ptx::umma_commit(kempty(k % KS));
+            ++k;
+            cg[gq] = c + 1;
+            if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
+          }
+          if (!ptx::mbar_wait(s_empty + 8u * (ti & 1), ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
+          ptx::tc_fence_after();
+          const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            ptx::umma_bf16(tS + (ti & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
+                           qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
+          }
+          ptx::umma_commit(s_full + 8u * (ti & 1));
+          ptx::umma_commit(kempty(k % KS));        // the K slot is free once S is done
+          ++k;
+        }
+        // every MMA issued so far must finish before tensor memory is released
+        ptx::umma_commit(drain_bar);
+        volatile int never = 0;
+        ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
+      } else {
+        constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
+        constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
+        // Base descriptors; every MMA operand below is one of these plus a
+        // constant byte offset (the address field is the low 14 bits, >> 4).
+        const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
+        const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
+        const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + KC::oV, kHalfTileBytes, 1024);  // V^T, MN-major
+        const uint64_t pdesc0 = ptx::sdesc_noswz(sP0, 16 * 2 * N, 128);              // [P_hi; P_lo], MN-major
+        int k = 0, i = 0;                        // K-ring items, tiles issued
+        int cg[2] = {0, 0};                      // chunks issued per group
+        PlanState ps0(p.nl), ps1(p.nl);
+        bool ok = true;
+        auto issue_pv = [&](int j) -> bool {
+          if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
+          if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
+          if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
+          ptx::tc_fence_after();
+          const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
+          const uint64_t pbd = pdesc0 + (uint64_t)(((j % KC::kPBufs) * KC::kPBufBytes) >> 4);
+          // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            ptx::umma_bf16(tO + (j & 1) * 2 * N, va + (uint64_t)((kk * 2048) >> 4),
+                           pbd + (uint64_t)((kk * (2 * 16 * 2 * N)) >> 4), kIdescPV, kk > 0);
+          }
+          ptx::umma_commit(o_full + 8u * (j & 1));
+          ptx::umma_commit(vempty(j % VS));
+          return true;
+        };
+        for (int ti = 0; ti < g.ntiles; ++ti) {
+          const int gq = KC::kAlt ? (ti & 1) : 0;
+          const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
+          // P.V of the previous tile frees a V slot: issue it first unless this
+          // tile's K data has already landed (then S first, so softmax starts).
+          bool pv_pending = i > 0;
+          if (pv_pending) {
+            const int kt = k + (tp.chunk ? 1 : 0);
+            if (!ptx::mbar_try_wait(kfull(kt % KS), (kt / KS) & 1)) {
+              if (!(ok = issue_pv(i - 1))) break;
+              pv_pending = false;
+            }
+          }
+          if (tp.chunk) {
+            const int c = cg[gq];
+            ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
+                 ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
+              const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+              ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
+              if constexpr (ROWS > 128)
+                ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
+            }
+            ptx::umma_commit(x_full + 8u * gq);
+            ptx::umma_commit(kempty(k % KS));
+            ++k;
+            cg[gq] = c + 1;
+          }
+          ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
+               ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          {
+            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              ptx::umma_bf16(tS + (i & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
+                             qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
+            }
+            ptx::umma_commit(s_full + 8u * (i & 1));
+            ptx::umma_commit(kempty(k % KS));      // the K slot is free once S is done
+          }
+          if (pv_pending && !(ok = issue_pv(i - 1))) break;
+          ++k;
+          ++i;
+        }
+        if (ok && i > 0) ok = issue_pv(i - 1);
+        // every MMA issued so far must finish before tensor memory is released
+        ptx::umma_commit(drain_bar);
+        volatile int never = 0;
+        ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
+      }
+    }
+    __syncwarp();
+  }
+  // ----------------------------------------------------------- P.V issuer
+  else if (KC::kSplitIssue && warp == KC::kPvWarp) {
+    if (lane == 0) {
       constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
-      // Base descriptors; every MMA operand below is one of these plus a
-      // constant byte offset (the address field is the low 14 bits, >> 4).
-      const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
-      const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
       const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + KC::oV, kHalfTileBytes, 1024);  // V^T, MN-major
       const uint64_t pdesc0 = ptx::sdesc_noswz(sP0, 16 * 2 * N, 128);              // [P_hi; P_lo], MN-major
-      int k = 0, i = 0;                        // K-ring items, tiles issued
-      int cg[2] = {0, 0};                      // chunks issued per group
-      PlanState ps0(p.nl), ps1(p.nl);
-      bool ok = true;
-      auto issue_pv = [&](int j) -> bool {
-        if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
-        if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
-        if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
+      for (int j = 0; j < g.ntiles; ++j) {
+        if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim) ||
+            !ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim) ||
+            !ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim))
+          break;
         ptx::tc_fence_after();
         const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
         const uint64_t pbd = pdesc0 + (uint64_t)(((j % KC::kPBufs) * KC::kPBufBytes) >> 4);
@@ -686,64 +841,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         }
         ptx::umma_commit(o_full + 8u * (j & 1));
         ptx::umma_commit(vempty(j % VS));
-        return true;
-      };
-      for (int ti = 0; ti < g.ntiles; ++ti) {
-        const int gq = KC::kAlt ? (ti & 1) : 0;
-        const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
-        // P.V of the previous tile frees a V slot: issue it first unless this
-        // tile's K data has already landed (then S first, so softmax starts).
-        bool pv_pending = i > 0;
-        if (pv_pending) {
-          const int kt = k + (tp.chunk ? 1 : 0);
-          if (!ptx::mbar_try_wait(kfull(kt % KS), (kt / KS) & 1)) {
-            if (!(ok = issue_pv(i - 1))) break;
-            pv_pending = false;
-          }
-        }
-        if (tp.chunk) {
-          const int c = cg[gq];
-          ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
-               ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
-            const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
-            ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
-            if constexpr (ROWS > 128)
-              ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
-          }
-          ptx::umma_commit(x_full + 8u * gq);
-          ptx::umma_commit(kempty(k % KS));
-          ++k;
-          cg[gq] = c + 1;
-        }
-        ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
-             ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        {
-          const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            ptx::umma_bf16(tS + (i & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
-                           qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
-          }
-          ptx::umma_commit(s_full + 8u * (i & 1));
-          ptx::umma_commit(kempty(k % KS));      // the K slot is free once S is done
-        }
-        if (pv_pending && !(ok = issue_pv(i - 1))) break;
-        ++k;
-        ++i;
       }
-      if (ok && i > 0) ok = issue_pv(i - 1);
-      // every MMA issued so far must finish before tensor memory is released
-      ptx::umma_commit(drain_bar);
+      ptx::umma_commit(drain_pv);
       volatile int never = 0;
-      ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
+      ptx::mbar_wait(drain_pv, 0, &never, kDrainLimitNs);
     }
     __syncwarp();
   }
