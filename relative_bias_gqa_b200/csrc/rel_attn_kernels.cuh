@@ -699,7 +699,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             if (!ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim)) break;
             ptx::tc_fence_after();
             const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
               const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
@@ -716,7 +716,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           if (!ptx::mbar_wait(s_empty + 8u * (ti & 1), ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
           ptx::tc_fence_after();
           const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             ptx::umma_bf16(tS + (ti & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
                            qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
@@ -750,7 +750,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
           const uint64_t pbd = pdesc0 + (uint64_t)(((j % KC::kPBufs) * KC::kPBufBytes) >> 4);
           // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             ptx::umma_bf16(tO + (j & 1) * 2 * N, va + (uint64_t)((kk * 2048) >> 4),
                            pbd + (uint64_t)((kk * (2 * 16 * 2 * N)) >> 4), kIdescPV, kk > 0);
@@ -779,7 +779,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             if (!ok) break;
             ptx::tc_fence_after();
             const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
               const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
@@ -798,7 +798,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           ptx::tc_fence_after();
           {
             const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               ptx::umma_bf16(tS + (i & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
                              qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
