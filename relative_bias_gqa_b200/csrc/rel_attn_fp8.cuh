@@ -407,7 +407,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
     for (int r = 0; r < RG; ++r) { l_part[r] = 0.f; o_acc[r] = 0.f; m_ref[r] = kNoMax; alpha_r[r] = 1.f; }
     int c = 0, li = 0;
-    PlanState ps0(p.nl), ps1(p.nl);
+    PlanState ps(p.nl);                       // this group's tiles only
     bool failed = false, aborted = false;
 
     // O^T of tile j: columns 0..G-1 from P_hi, G..2G-1 from P_mid, 2G..3G-1
@@ -431,11 +431,17 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       if (!okw) failed = true;
     };
 
-    for (int ti = 0; ti < g.ntiles; ++ti) {
-      const int owner = ti & 1;
-      const TilePlan tp = plan_tile<128>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, owner ? ps1 : ps0);
-      const int c0 = owner ? ps1.c0 : ps0.c0;
-      if (owner != grp) continue;
+    // Group g takes the tiles g, g + 2, ...; the plan of its next tile is
+    // made while P.V of the current one runs.
+    TilePlan tp_next{};
+    int c0_next = 0;
+    if (grp < g.ntiles) {
+      tp_next = plan_tile<128>(g, grp, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
+      c0_next = ps.c0;
+    }
+    for (int ti = grp; ti < g.ntiles; ti += 2) {
+      const TilePlan tp = tp_next;
+      const int c0 = c0_next;
       if (tp.chunk) {
         // ---- new relative-row chunk: X^T (128 rows x G) -> gather table Y
         const bool okw = ptx::mbar_wait(x_full + 8u * grp, c & 1, abort_flag, tlim);
@@ -565,6 +571,10 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
+      if (ti + 2 < g.ntiles) {
+        tp_next = plan_tile<128>(g, ti + 2, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
+        c0_next = ps.c0;
+      }
       process_o(i);                            // this group's next tile is i + 2
       ++li;
     }

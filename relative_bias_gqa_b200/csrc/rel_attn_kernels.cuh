@@ -906,7 +906,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
     for (int r = 0; r < (KC::kAlt ? RG : 1); ++r) alpha_r[r] = 1.f;
     int c = 0, li = 0;                        // own chunks, own tiles
-    PlanState ps0(p.nl), ps1(p.nl);
+    PlanState ps(p.nl);                       // planned over this group's tiles
     bool failed = false, aborted = false;
 
     // Accumulate the O^T tile of tile j (this thread's head-dim lane, this
@@ -931,13 +931,26 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     };
 
     int last_tile = -1;
-    for (int ti = 0; ti < g.ntiles; ++ti) {
-      const int owner = KC::kAlt ? (ti & 1) : grp;
-      const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges,
-                                          (KC::kAlt && owner) ? ps1 : ps0);
-      const int c0 = (KC::kAlt && owner) ? ps1.c0 : ps0.c0;
+    // This group's tiles: every other one (alternating groups) or all.  With
+    // alternating groups the plan of the group's next tile is made while P.V
+    // of the current one runs (elsewhere the registers are scarcer).
+    constexpr int kStep = KC::kAlt ? 2 : 1;
+    const int t_first = KC::kAlt ? grp : 0;
+    TilePlan tp_next{};
+    int c0_next = 0;
+    if (KC::kAlt && t_first < g.ntiles) {
+      tp_next = plan_tile<ROWS>(g, t_first, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
+      c0_next = ps.c0;
+    }
+    for (int ti = t_first; ti < g.ntiles; ti += kStep) {
+      TilePlan tp = tp_next;
+      int c0 = c0_next;
+      if constexpr (!KC::kAlt) {
+        tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
+        c0 = ps.c0;
+      }
       if (tp.chunk) {
-        if (owner == grp) {
+        {
           // ---- new relative-row chunk: this group's columns of X^T (128 or
           //      136 relative rows) -> gather table Y
           const int xb = KC::kAlt ? grp : 0;
@@ -964,7 +977,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
         }
       }
-      if (owner != grp) continue;
       const int i = ti;                       // buffers and phases follow the tile index
 
       // ---- S^T tile: this thread owns key j, this group's columns
@@ -1120,6 +1132,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
+      if (KC::kAlt && ti + kStep < g.ntiles) {
+        tp_next = plan_tile<ROWS>(g, ti + kStep, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
+        c0_next = ps.c0;
+      }
       if constexpr (KC::kAlt) {
         // this group's next tile is i + 2: take O(i) now
         process_o(i, alpha_r);
