@@ -16,9 +16,10 @@
 //   O^T = V8^T . [P_hi; P_mid; P_lo]^T   P = P_hi + P_mid / 16 + P_lo / 256,
 //                                   12 significant bits
 //   X^T = R_chunk . Q^T             bf16 (kind::f16) as in the bf16 kernel
-// Roles: warp 0 TMA producer (K8 and V8 page tiles, 8 KB per page, and
-// relative-row chunks, each in its own ring), warp 1 issues S and X, warp 10
-// issues P.V, two softmax groups of 4 warps (2..9) alternate tiles.  The two
+// Roles: warp 0 TMA producer of K8 page tiles (8 KB per page) and
+// relative-row chunks, warp 11 of V8 page tiles (each in its own ring), warp
+// 1 issues S and X, warp 10 issues P.V, two softmax groups of 4 warps (2..9)
+// alternate tiles.  The two
 // MMA issuers run side by side: a single issuing thread spends about a
 // microsecond per tile on its waits, descriptors and eight MMA issues, more
 // than the tile's bytes take to arrive at the HBM rate.
@@ -36,7 +37,8 @@ struct Fp8Config {
   static constexpr int NG = 2, RG = G;
   static_assert(2 * G <= N && 3 * G <= NP && G % 2 == 0, "group size");
   static constexpr int kPvWarp = 2 + 4 * NG;                   // after the softmax warps
-  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + 32;
+  static constexpr int kVWarp = kPvWarp + 1;                    // V-tile producer
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + 64;
   static constexpr int kKSlots = 4, kVSlots = 6, kRSlots = 1;
   static constexpr int kTile8 = 128 * 128;                      // 128 keys x 128 B
   static constexpr int kPage8 = 64 * 128;
@@ -181,7 +183,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   }
   __syncthreads();
   uint32_t tmem = 0;
-  if (warp != 0) {
+  if (warp != 0 && warp != FC::kVWarp) {
     if (warp == 1) {
       ptx::tmem_alloc(ptx::smem_addr(tmem_holder), FC::kTmemCols);
       ptx::tmem_relinquish();
@@ -240,7 +242,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       ptx::fence_proxy_async_smem();
     }
     ptx::tc_fence_before();
-    ptx::bar_sync_or(kBarSetup, FC::kThreads - 32, false);   // every warp but the producer
+    ptx::bar_sync_or(kBarSetup, FC::kThreads - 64, false);   // every warp but the producers
     ptx::tc_fence_after();
     tmem = *tmem_holder;
   }
@@ -258,7 +260,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     };
     int bt_cur = bt_load(0);
     int bt_next = bt_load(1);
-    int nk = 0, nv = 0, nr = 0;                // K tiles, V tiles, relative chunks issued
+    int nk = 0, nr = 0;                        // K tiles, relative chunks issued
     PlanState ps0(p.nl), ps1(p.nl);
     bool ok = true, bad_page = false;
     for (int ti = 0; ti < g.ntiles; ++ti) {
@@ -294,20 +296,51 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         if (tp.npg > 1) ptx::tma_load_2d(kslot(ti) + FC::kPage8, &p.tmap_k, kfull(ti % KS), 0, row1, pol);
       }
       ++nk;
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(vempty(ti % VS), ((ti / VS) & 1) ^ 1, abort_flag, tlim));
-      if (!ok) break;
+    }
+    if (lane == 0) {
+      if (bad_page) *bad_page_flag = 1;
+      issued[0] = nk;                        // for the drain at teardown
+      issued[2] = nr;
+    }
+  }
+  // ------------------------------------------------------- V-tile producer
+  // V tiles come from a warp of their own: one warp issuing K, V and the
+  // relative chunks, with the tile plan in between, took longer per tile than
+  // the tile's bytes take to arrive.
+  else if (warp == FC::kVWarp) {
+    const uint64_t pol = ptx::l2_policy_evict_first();
+    const int* bt_row = p.block_table + (size_t)b * p.max_pages;
+    auto bt_load = [&](int grp) -> int {
+      const int pg = g.sp_begin + 32 * grp + lane;
+      return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
+    };
+    int bt_cur = bt_load(0);
+    int bt_next = bt_load(1);
+    int nv = 0;                                // V tiles issued
+    bool bad_page = false;
+    for (int ti = 0; ti < g.ntiles; ++ti) {
+      if (ti > 0 && (ti & 15) == 0) {
+        bt_cur = bt_next;
+        bt_next = bt_load((ti >> 4) + 1);
+      }
+      const int npg = min(2, g.sp_end - (g.sp_begin + 2 * ti));
+      int e0 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti) & 31);
+      int e1 = __shfl_sync(0xffffffffu, bt_cur, (2 * ti + 1) & 31);
+      if (e0 < 0 || e0 >= p.num_pages) { bad_page = true; e0 = 0; }
+      if (npg > 1 && (e1 < 0 || e1 >= p.num_pages)) { bad_page = true; e1 = 0; }
+      const int row0 = (e0 * p.Hkv + h) * kPage, row1 = (e1 * p.Hkv + h) * kPage;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(vempty(ti % VS), ((ti / VS) & 1) ^ 1, abort_flag, tlim)))
+        break;
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(vfull(ti % VS), tp.npg * FC::kPage8);
+        ptx::mbar_arrive_expect_tx(vfull(ti % VS), npg * FC::kPage8);
         ptx::tma_load_2d(vslot(ti), &p.tmap_v, vfull(ti % VS), 0, row0, pol);
-        if (tp.npg > 1) ptx::tma_load_2d(vslot(ti) + FC::kPage8, &p.tmap_v, vfull(ti % VS), 0, row1, pol);
+        if (npg > 1) ptx::tma_load_2d(vslot(ti) + FC::kPage8, &p.tmap_v, vfull(ti % VS), 0, row1, pol);
       }
       ++nv;
     }
     if (lane == 0) {
       if (bad_page) *bad_page_flag = 1;
-      issued[0] = nk;                        // for the drain at teardown
-      issued[1] = nv;
-      issued[2] = nr;
+      issued[1] = nv;                        // for the drain at teardown
     }
   }
   // ------------------------------------------------------- S and X issuer
