@@ -327,6 +327,13 @@ int rel_attn_bucket(const rel_attn_shape* shape, int distance);
 int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
                          int split, int* first_page, int* end_page);
 
+/* The same for the E4M3 kernel (rel_attn_decode_e4m3 / rel_attn_partial_e4m3),
+ * whose partition weighs an exact-range page more: such a tile also reads a
+ * 32 KB bf16 relative-row chunk, twice its E4M3 K and V bytes.  Arguments,
+ * results and errors as rel_attn_split_pages. */
+int rel_attn_split_pages_e4m3(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                              int split, int* first_page, int* end_page);
+
 /* Static description of an error code. */
 const char* rel_attn_error_string(int code);
 

@@ -392,8 +392,8 @@ int rel_attn_bucket(const rel_attn_shape* shape, int distance) {
   return bucket_host(distance, ex, nl, edges);
 }
 
-int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
-                         int split, int* first_page, int* end_page) {
+static int split_pages_api(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                           int split, int cost_exact, int* first_page, int* end_page) {
   if (validate_shape(shape) != REL_ATTN_OK || !first_page || !end_page) return REL_ATTN_ERR_INVALID_ARG;
   if (seq_len < shape->q_tokens || seq_len > shape->max_pages_per_seq * kPage)
     return REL_ATTN_ERR_INVALID_ARG;
@@ -404,8 +404,21 @@ int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, i
   bucket_table_cached(shape, &ex, &nl, edges);
   const int p0 = seq_len - shape->q_tokens;
   const int lo = (window > 0) ? std::max(0, p0 - window + 1) : 0;
-  split_pages(lo / kPage, (seq_len - 1) / kPage, num_splits, split, ex, first_page, end_page);
+  split_pages(lo / kPage, (seq_len - 1) / kPage, num_splits, split, ex, cost_exact, first_page,
+              end_page);
   return REL_ATTN_OK;
+}
+
+int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                         int split, int* first_page, int* end_page) {
+  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactBf16, first_page,
+                         end_page);
+}
+
+int rel_attn_split_pages_e4m3(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
+                              int split, int* first_page, int* end_page) {
+  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactE4m3, first_page,
+                         end_page);
 }
 
 int rel_attn_set_wait_limit(unsigned long long limit_ns) {
@@ -496,6 +509,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->window = window;
   prm->out_fp32 = shape->out_fp32;
   bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges, &prm->log2_ex, &prm->log_scale);
+  prm->cost_exact = kv_e4m3 ? kCostExactE4m3 : kCostExactBf16;
   prm->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
   prm->k_scale = k_scale;
   prm->v_scale = v_scale;

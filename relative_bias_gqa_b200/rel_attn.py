@@ -29,6 +29,7 @@ EXPORTED = (
     "rel_attn_error_string", "rel_attn_version", "rel_attn_decode_static",
     "rel_attn_split_pages", "rel_attn_decode_e4m3", "rel_attn_partial_e4m3",
     "rel_attn_set_wait_limit", "rel_attn_kv_write", "rel_attn_prefill",
+    "rel_attn_split_pages_e4m3",
 )
 
 
@@ -79,6 +80,8 @@ def _load():
     lib.rel_attn_split_pages.argtypes = [SP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.rel_attn_split_pages.restype = ctypes.c_int
+    lib.rel_attn_split_pages_e4m3.argtypes = lib.rel_attn_split_pages.argtypes
+    lib.rel_attn_split_pages_e4m3.restype = ctypes.c_int
     lib.rel_attn_prefill.argtypes = lib.rel_attn_decode.argtypes
     lib.rel_attn_prefill.restype = ctypes.c_int
     lib.rel_attn_kv_write.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, P, P]
@@ -139,11 +142,13 @@ def rel_attn_bucket(shape: RelAttnShape, distance: int) -> int:
 
 
 def rel_attn_split_pages(shape: RelAttnShape, seq_len: int, window: int, num_splits: int,
-                         split: int):
-    """(first_page, end_page) of one split, as the partial kernel walks it."""
+                         split: int, e4m3: bool = False):
+    """(first_page, end_page) of one split, as the partial kernel (the E4M3
+    one with e4m3=True) walks it."""
     a, b = ctypes.c_int(), ctypes.c_int()
-    rc = lib.rel_attn_split_pages(ctypes.byref(shape), int(seq_len), int(window), int(num_splits),
-                                  int(split), ctypes.byref(a), ctypes.byref(b))
+    fn = lib.rel_attn_split_pages_e4m3 if e4m3 else lib.rel_attn_split_pages
+    rc = fn(ctypes.byref(shape), int(seq_len), int(window), int(num_splits),
+            int(split), ctypes.byref(a), ctypes.byref(b))
     if rc != REL_ATTN_OK:
         raise RelAttnError(rc)
     return a.value, b.value

@@ -198,7 +198,8 @@ def test_error_strings(ra):
 @pytest.mark.parametrize("L,T,window,nb", [(100_000, 1, 0, 1280), (262_144, 8, 0, 1280),
                                             (100_000, 1, 1024, 1024), (20_000, 3, 0, 1280),
                                             (5, 1, 0, 1280), (2048, 2, 100, 364)])
-def test_split_pages_partition(ra, L, T, window, nb):
+@pytest.mark.parametrize("e4m3", [False, True])
+def test_split_pages_partition(ra, L, T, window, nb, e4m3):
     """Every split count gives contiguous, ordered page ranges that cover
     exactly the pages some query can see, tiles stay two pages long inside,
     and near-query splits are no longer than far ones."""
@@ -211,7 +212,7 @@ def test_split_pages_partition(ra, L, T, window, nb):
         prev = first
         sizes = []
         for sp in range(S):
-            a, b = ra.rel_attn_split_pages(s, L, window, S, sp)
+            a, b = ra.rel_attn_split_pages(s, L, window, S, sp, e4m3=e4m3)
             assert a == prev and b >= a
             assert (a - first) % 2 == 0 or a == last + 1      # inner boundaries keep 2-page tiles
             sizes.append(b - a)
@@ -222,13 +223,27 @@ def test_split_pages_partition(ra, L, T, window, nb):
             assert big[-1] <= max(big[:-1])
 
 
-def test_split_pages_rejects_bad_arguments(ra):
+@pytest.mark.parametrize("name", ["rel_attn_split_pages", "rel_attn_split_pages_e4m3"])
+def test_split_pages_rejects_bad_arguments(ra, name):
     s = shape(ra)
     import ctypes
     a, b = ctypes.c_int(), ctypes.c_int()
-    f = ra.lib.rel_attn_split_pages
+    f = getattr(ra.lib, name)
     assert f(ctypes.byref(s), 100, 0, 4, 4, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
     assert f(ctypes.byref(s), 100, 0, 0, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
     assert f(ctypes.byref(s), 0, 0, 4, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
     assert f(ctypes.byref(s), 1 << 30, 0, 4, 0, ctypes.byref(a), ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
     assert f(ctypes.byref(s), 100, 0, 4, 0, None, ctypes.byref(b)) == ra.REL_ATTN_ERR_INVALID_ARG
+
+
+def test_e4m3_partition_gives_the_exact_range_fewer_pages(ra):
+    """The E4M3 weights put fewer pages in the split nearest the queries
+    (its tiles carry a relative-row chunk twice their K/V bytes)."""
+    L = 100_000
+    pages = (L + 63) // 64 + 1
+    s = shape(ra, q_tokens=1, num_buckets=1280, max_pages_per_seq=pages, num_pages=pages,
+              max_seq_len=L, exact_buckets=1024)
+    a16, b16 = ra.rel_attn_split_pages(s, L, 0, 18, 17)
+    a8, b8 = ra.rel_attn_split_pages(s, L, 0, 18, 17, e4m3=True)
+    assert b16 == b8 == (L - 1) // 64 + 1
+    assert b8 - a8 < b16 - a16
