@@ -110,6 +110,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
+  // the block-table row towards L2 while the length is read
+  if (warp == 0)
+    ptx::prefetch_l2_range(p.block_table + (size_t)b * p.max_pages, (size_t)p.max_pages * 4, 128, lane);
   g.L = __ldg(p.seq_lens + b);
   g.T = T;
   if (g.L < T || g.L > p.max_pages * kPage) {

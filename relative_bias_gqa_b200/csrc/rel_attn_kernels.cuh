@@ -466,6 +466,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   // ------------------------------------------------------------ geometry
   const int row0 = first_token_row(p, b);      // q / out row of query token 0
   const int b_seq = b / p.cps;                 // the sequence (block-table row)
+  // the block-table row towards L2 while the length is read: the split's
+  // entries follow from it, and the producer's first load then hits L2
+  if (warp == 0)
+    ptx::prefetch_l2_range(p.block_table + (size_t)b_seq * p.max_pages, (size_t)p.max_pages * 4, 128, lane);
   SplitGeom g;
   // the sequence must hold all of its query tokens (seq_stride of them: T
   // for a decode step, C for a prefill) and fit its block-table row
@@ -1290,6 +1294,18 @@ rel_attn_combine_kernel(const float* __restrict__ ws_lse, const float* __restric
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int row = blockIdx.x;
   const float l = (t < num_splits) ? __ldg(ws_lse + (size_t)t * rows + row) : -INFINITY;
+  // this warp's first kPre splits' partial outputs, in flight while the
+  // weights are formed (the workspace holds every split's row, empty splits
+  // included, so these loads stay inside it)
+  constexpr int kPre = 4;
+  float4 opre[kPre];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    const int s = warp + 8 * k;
+    opre[k] = (s < num_splits)
+                  ? __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)s * rows + row) * kHeadDim) + lane)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (__syncthreads_or(l != l)) {                  // a rejected sequence: propagate NaN
     if (t < 32) {
       const float qnan = __int_as_float(0x7fc00000);
@@ -1316,7 +1332,18 @@ rel_attn_combine_kernel(const float* __restrict__ ws_lse, const float* __restric
   __syncthreads();                                   // w_s complete, red[] reads done
   if (lane == 0) red[warp] = sum;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = warp; s < num_splits; s += 8) {
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    const int s = warp + 8 * k;
+    const float ws = (s < num_splits) ? w_s[s] : 0.f;
+    if (ws != 0.f) {
+      acc.x = fmaf(ws, opre[k].x, acc.x);
+      acc.y = fmaf(ws, opre[k].y, acc.y);
+      acc.z = fmaf(ws, opre[k].z, acc.z);
+      acc.w = fmaf(ws, opre[k].w, acc.w);
+    }
+  }
+  for (int s = warp + 8 * kPre; s < num_splits; s += 8) {
     const float ws = w_s[s];
     if (ws != 0.f) {
       const float4 o = __ldg(reinterpret_cast<const float4*>(ws_o + ((size_t)s * rows + row) * kHeadDim) + lane);

@@ -98,6 +98,18 @@ __device__ __forceinline__ bool bar_sync_or(int id, int nthreads, bool pred) {
 }
 
 // ---------------------------------------------------------------------- TMA
+// L2 prefetch of the 128-byte lines that hold [ptr, ptr + bytes), one line
+// per lane of the calling warp (lines that hold no byte of the range are not
+// touched); nothing if the range spans more than `max_lines` lines.
+__device__ __forceinline__ void prefetch_l2_range(const void* ptr, size_t bytes, int max_lines, int lane) {
+  if (bytes == 0) return;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(ptr);
+  const uintptr_t first = a >> 7, last = (a + bytes - 1) >> 7;
+  if (last - first + 1 > (uintptr_t)max_lines) return;
+  for (uintptr_t line = first + lane; line <= last; line += 32)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(line << 7));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
