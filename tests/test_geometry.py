@@ -65,7 +65,7 @@ def test_inkling2_instances(table):
     # 48/8 heads: N and group counts of the measured instances; nine tokens
     # (an 8-head MTP chain's verify step) need the 64-wide instance
     assert [table[(6, t)][0] for t in range(1, 10)] == [16, 32, 32, 32, 48, 48, 64, 64, 64]
-    assert [table[(6, t)][1] for t in range(1, 10)] == [2, 2, 2, 2, 2, 4, 4, 4, 4]
+    assert [table[(6, t)][1] for t in range(1, 10)] == [2, 2, 2, 2, 2, 4, 4, 4, 3]
     # 7 and 8 tokens: 8-aligned blocks in the 64-wide tile; 9 tokens 4-aligned
     assert [table[(6, t)][2] for t in range(6, 10)] == [8, 8, 8, 4]
 
@@ -73,8 +73,10 @@ def test_inkling2_instances(table):
 def test_wide_instances(table):
     # 64/8 heads with 7 and 8 tokens: four groups of up to 16 rows, 8-aligned
     assert [table[(8, t)][:3] for t in (7, 8)] == [(64, 4, 8), (64, 4, 8)]
-    # nine tokens over four groups: 2/2/2/3 tokens, the last group 18 rows
-    assert [g[2] for g in table[(6, 9)][3]] == [12, 12, 12, 18]
+    # nine tokens at G = 6: three groups of three tokens, 18 rows each at
+    # 4-aligned query slots 0 / 20 / 40
+    assert [g[2] for g in table[(6, 9)][3]] == [18, 18, 18]
+    assert [g[1] for g in table[(6, 9)][3]] == [0, 20, 40]
     assert table[(4, 9)][:2] == (48, 4)
 
 
