@@ -65,7 +65,7 @@ def test_inkling2_instances(table):
     # 48/8 heads: N and group counts of the measured instances; nine tokens
     # (an 8-head MTP chain's verify step) need the 64-wide instance
     assert [table[(6, t)][0] for t in range(1, 10)] == [16, 32, 32, 32, 48, 48, 64, 64, 64]
-    assert [table[(6, t)][1] for t in range(1, 10)] == [2, 2, 2, 2, 2, 4, 4, 4, 3]
+    assert [table[(6, t)][1] for t in range(1, 10)] == [2, 2, 2, 2, 2, 3, 4, 4, 3]
     # 7 and 8 tokens: 8-aligned blocks in the 64-wide tile; 9 tokens 4-aligned
     assert [table[(6, t)][2] for t in range(6, 10)] == [8, 8, 8, 4]
 
