@@ -393,7 +393,8 @@ int rel_attn_bucket(const rel_attn_shape* shape, int distance) {
 }
 
 static int split_pages_api(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
-                           int split, int cost_exact, int* first_page, int* end_page) {
+                           int split, int cost_exact, int cost_near, int* first_page,
+                           int* end_page) {
   if (validate_shape(shape) != REL_ATTN_OK || !first_page || !end_page) return REL_ATTN_ERR_INVALID_ARG;
   if (seq_len < shape->q_tokens || seq_len > shape->max_pages_per_seq * kPage)
     return REL_ATTN_ERR_INVALID_ARG;
@@ -404,21 +405,21 @@ static int split_pages_api(const rel_attn_shape* shape, int seq_len, int window,
   bucket_table_cached(shape, &ex, &nl, edges);
   const int p0 = seq_len - shape->q_tokens;
   const int lo = (window > 0) ? std::max(0, p0 - window + 1) : 0;
-  split_pages(lo / kPage, (seq_len - 1) / kPage, num_splits, split, ex, cost_exact, first_page,
-              end_page);
+  split_pages(lo / kPage, (seq_len - 1) / kPage, num_splits, split, ex, cost_exact, cost_near,
+              first_page, end_page);
   return REL_ATTN_OK;
 }
 
 int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
                          int split, int* first_page, int* end_page) {
-  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactBf16, first_page,
-                         end_page);
+  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactBf16, kCostNearBf16,
+                         first_page, end_page);
 }
 
 int rel_attn_split_pages_e4m3(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
                               int split, int* first_page, int* end_page) {
-  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactE4m3, first_page,
-                         end_page);
+  return split_pages_api(shape, seq_len, window, num_splits, split, kCostExactE4m3, kCostNearE4m3,
+                         first_page, end_page);
 }
 
 int rel_attn_set_wait_limit(unsigned long long limit_ns) {
@@ -510,6 +511,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->out_fp32 = shape->out_fp32;
   bucket_table_cached(shape, &prm->ex, &prm->nl, prm->edges, &prm->log2_ex, &prm->log_scale);
   prm->cost_exact = kv_e4m3 ? kCostExactE4m3 : kCostExactBf16;
+  prm->cost_near = kv_e4m3 ? kCostNearE4m3 : kCostNearBf16;
   prm->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
   prm->k_scale = k_scale;
   prm->v_scale = v_scale;

@@ -123,7 +123,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   g.p0 = g.L - T;
   g.W = p.window;
   g.lo = (g.W > 0) ? max(0, g.p0 - g.W + 1) : 0;
-  split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, p.cost_exact, &g.sp_begin,
+  split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, p.cost_exact, p.cost_near, &g.sp_begin,
               &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {

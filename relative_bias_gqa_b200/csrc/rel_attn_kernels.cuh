@@ -111,7 +111,8 @@ struct alignas(64) DecodeParams {
   int cps, seq_stride, tok_off, len_off;
   int rows_total;       // rows of the partial buffers: all query tokens x Hq
   int ex;               // distances d < ex are their own bucket
-  int cost_exact;       // split weight of an exact-range page (see split_pages)
+  int cost_exact;       // split weights of an exact-range and a narrow-bucket
+  int cost_near;        // page (see split_pages)
   int nl;               // tail buckets: bucket = ex + max{k < nl : edges[k] <= d}
   float scale_log2;     // log2(e) / sqrt(D)
   float log2_ex, log_scale;  // tail-bucket guess: (log2(d) - log2_ex) * log_scale
@@ -322,7 +323,7 @@ __device__ __forceinline__ int step_down(int k, int d, const int* edges, float l
 // exact-distance range every tile needs its own relative-row chunk, and up
 // to a few thousand keys out the tail buckets are narrow), so the page at
 // distance rank q from the query end is weighted 8 + cost_exact [q < QE] +
-// kCostNear [q < QN] eighths.  The cumulative cost from the query end is
+// cost_near [q < QN] eighths.  The cumulative cost from the query end is
 // piecewise linear and is inverted per boundary; interior boundaries are
 // rounded to an even page offset so that tiles stay two pages long.  The
 // exact-range weight depends on the cache type: an exact-range tile also
@@ -331,14 +332,17 @@ __device__ __forceinline__ int step_down(int k, int d, const int* edges, float l
 // Chosen on B200 by timing 100K-key batch-1 decode at 48/8 and 64/8 heads
 // over 18 splits: bf16 3, 4 and 5 time alike; E4M3 8 / 11 / 14 / 17 / 21
 // give 55.4 / 54.3 / 52.5 / 51.5 / 51.8 us per call at 48/8 heads (21 and
-// more lose at 64/8).
-constexpr int kCostExactBf16 = 5, kCostExactE4m3 = 17, kCostNear = 1;
+// more lose at 64/8); an E4M3 narrow-bucket weight of 2 then brings 64/8
+// from 52.1 to 50.2 us (48/8 unchanged).
+constexpr int kCostExactBf16 = 5, kCostNearBf16 = 1;
+constexpr int kCostExactE4m3 = 17, kCostNearE4m3 = 2;
 __host__ __device__ __forceinline__ void split_pages(int first, int last, int S, int s, int ex,
-                                                     int cost_exact, int* begin, int* end) {
+                                                     int cost_exact, int cost_near, int* begin,
+                                                     int* end) {
   const int n = last - first + 1;
   const int qe = min(n, (ex + 128 + kPage - 1) / kPage + 1);   // pages holding exact-range keys
   const int qn = min(n, max(qe, 8 * ex / kPage));              // pages of the narrow tail buckets
-  const int s1 = 8 + cost_exact + kCostNear, s2 = 8 + kCostNear;
+  const int s1 = 8 + cost_exact + cost_near, s2 = 8 + cost_near;
   const int ce = s1 * qe;                                      // cost of the first qe pages
   const int cn = ce + s2 * (qn - qe);                          // ... of the first qn pages
   const int total = cn + 8 * (n - qn);                         // < 2^31 for n < 2^27 pages
@@ -490,7 +494,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   g.p0 = g.L - T;
   g.W = p.window;
   g.lo = (g.W > 0) ? max(0, g.p0 - g.W + 1) : 0;
-  split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, p.cost_exact, &g.sp_begin,
+  split_pages(g.lo / kPage, (g.L - 1) / kPage, p.num_splits, s_idx, p.ex, p.cost_exact, p.cost_near, &g.sp_begin,
               &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {                       // a trailing split with no page
