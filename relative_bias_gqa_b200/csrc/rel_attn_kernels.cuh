@@ -60,12 +60,14 @@ constexpr int kBarSetup = 6;                   // every warp but the producer (p
 // softmax warps to hide each other's latencies), and always past 48 query
 // rows (the 64-wide instances); else two.
 __host__ __device__ constexpr int softmax_groups(int G, int T) {
-  // Six and nine tokens at G = 6: three groups of two / three tokens (12 or
-  // 18 rows each).  On the 256K verify step: 221 against 265 us (four groups,
-  // 1 / 2 / 1 / 2 tokens) and 374 against 501 us (2 / 2 / 2 / 3).  Uneven
-  // thirds lose: 7 and 8 tokens took 368 and 377 us with three groups against
-  // 258 and 247 with four, and 7 tokens at G = 8 205 against 199.
-  if (G == 6 && T >= 6 && T % 3 == 0) return 3;
+  // Six and nine tokens: three groups of two / three tokens.  On the 256K
+  // verify step at G = 6: 221 against 265 us (four groups, 1 / 2 / 1 / 2
+  // tokens) and 374 against 501 us (2 / 2 / 2 / 3); on 100K keys at G = 8
+  // with six tokens 118 against 130 us (two groups), at G = 4 with six and
+  // nine 159 and 177 against 171 and 197 us (four groups).  Uneven thirds
+  // lose: 7 and 8 tokens at G = 6 took 368 and 377 us with three groups
+  // against 258 and 247 with four, 7 at G = 8 205 against 199.
+  if (T >= 6 && T % 3 == 0) return 3;
   return (T >= 6 && ((T + 3) / 4 * G <= 12 || G * T > 48)) ? 4 : 2;
 }
 constexpr int kVSlotBytes = 32768;             // V tile: 128 keys x 128 dims bf16

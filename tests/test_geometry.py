@@ -77,7 +77,10 @@ def test_wide_instances(table):
     # 4-aligned query slots 0 / 20 / 40
     assert [g[2] for g in table[(6, 9)][3]] == [18, 18, 18]
     assert [g[1] for g in table[(6, 9)][3]] == [0, 20, 40]
-    assert table[(4, 9)][:2] == (48, 4)
+    # nine tokens at G = 4: three groups of 12 rows, 8-aligned in 48 columns
+    assert table[(4, 9)][:3] == (48, 3, 8)
+    # six tokens: three groups of two tokens for every G
+    assert [table[(g, 6)][1] for g in (4, 6, 8)] == [3, 3, 3]
 
 
 @pytest.mark.parametrize("G,T", [k for k in SUPPORTED if k[1] >= 2])
