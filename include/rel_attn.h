@@ -157,7 +157,12 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
  * MMAs, fp32 accumulation): the query is carried as two E4M3 terms scaled
  * per row by a power of two (exact for a bf16 query), the softmax weights
  * as three (12 significant bits); the relative term stays bf16.
- * Current limits: shape->q_tokens must be 1 and Hq/Hkv must be 4, 6 or 8
+ * Several query tokens (a verify step, q_tokens 2..9) run as one-token chunks
+ * of each sequence, token t attending to the keys before position L - T + t
+ * + 1 as in rel_attn_decode; the chunks of one (split, KV head) are launched
+ * side by side so that their page reads meet in L2, but each does the
+ * one-token work, so T tokens cost about T one-token calls of compute.
+ * Limits: Hq/Hkv must be 4, 6 or 8 and the shape valid for rel_attn_decode
  * (else REL_ATTN_ERR_INVALID_ARG).
  */
 int rel_attn_decode_e4m3(const rel_attn_shape* shape, const void* q,

@@ -459,7 +459,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
   if (kv_e4m3) {
-    if (shape->q_tokens != 1 || !k_scale || !v_scale ||
+    if (!k_scale || !v_scale ||
         (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))
       return REL_ATTN_ERR_INVALID_ARG;
   }
@@ -487,7 +487,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
   if (!cached_map(&prm->tmap_k, kv_e4m3 ? 4 : 0, k_cache, kv_rows, 0) ||
       !cached_map(&prm->tmap_v, kv_e4m3 ? 5 : 1, v_cache, kv_rows, 0) ||
-      !cached_map(&prm->tmap_r, group_width_for(Hq / Hkv, T) == 16 ? 3 : 2, rel_table,
+      !cached_map(&prm->tmap_r, (kv_e4m3 || group_width_for(Hq / Hkv, T) == 16) ? 3 : 2, rel_table,
                   (uint64_t)shape->num_buckets, (uint64_t)Hkv))
     return REL_ATTN_ERR_CUDA;
   prm->q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -503,6 +503,12 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->timeout_ns = wl ? wl : kDefaultTimeoutNs;
   prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
   prm->cps = 1; prm->seq_stride = T; prm->tok_off = 0; prm->len_off = 0;
+  if (kv_e4m3 && T > 1) {
+    // the E4M3 kernel is a one-token kernel: T tokens run as T one-token
+    // chunks of the sequence, each attending causally up to its position
+    prm->T = 1;
+    prm->cps = T;
+  }
   prm->rows_total = (int)rows;
   prm->num_pages = shape->num_pages;
   prm->max_pages = shape->max_pages_per_seq;
@@ -542,7 +548,7 @@ int launch_partial_e4m3_g(const DecodeParams& prm, int S, int B, int Hkv, cudaSt
       return REL_ATTN_ERR_CUDA;
     attr = true;
   }
-  dim3 grid(S, Hkv, B);
+  dim3 grid(S * prm.cps, Hkv, B);                  // chunk index fastest in x
   kern<<<grid, FC::kThreads, FC::kAllocBytes, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? REL_ATTN_OK : REL_ATTN_ERR_CUDA;
 }

@@ -106,18 +106,26 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int s_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Several query tokens run as one-token chunks (DecodeParams::cps of them
+  // per sequence), the chunk index fastest in x so that the CTAs of one
+  // (split, KV head) read the same pages at about the same time.
+  const int chunk = (int)blockIdx.x % p.cps;
+  const int s_idx = (int)blockIdx.x / p.cps, h = blockIdx.y;
+  const int b_seq = blockIdx.z;                    // the sequence (block-table row)
+  const int b = b_seq * p.cps + chunk;             // grid z-index of this chunk
+  const int row0 = first_token_row(p, b);          // q / out row of its token
 
   // ------------------------------------------------------------ geometry
   SplitGeom g;
   // the block-table row towards L2 while the length is read
   if (warp == 0)
-    ptx::prefetch_l2_range(p.block_table + (size_t)b * p.max_pages, (size_t)p.max_pages * 4, 128, lane);
-  g.L = __ldg(p.seq_lens + b);
+    ptx::prefetch_l2_range(p.block_table + (size_t)b_seq * p.max_pages, (size_t)p.max_pages * 4, 128, lane);
+  const int L_seq = __ldg(p.seq_lens + b_seq);
+  g.L = chunk_seq_len(p, b, L_seq);
   g.T = T;
-  if (g.L < T || g.L > p.max_pages * kPage) {
+  if (L_seq < p.seq_stride || L_seq > p.max_pages * kPage) {
     if (tid == 0) atomicOr(p.status, kStatusBadSeq);
-    fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, row0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     return;
   }
   g.p0 = g.L - T;
@@ -127,7 +135,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
               &g.sp_end);
   g.ntiles = (g.sp_end > g.sp_begin) ? (g.sp_end - g.sp_begin + 1) / 2 : 0;
   if (g.ntiles == 0) {
-    fill_rows<G>(p, first_token_row(p, b), h, s_idx, 0.f, -INFINITY);
+    fill_rows<G>(p, row0, h, s_idx, 0.f, -INFINITY);
     return;
   }
 
@@ -201,7 +209,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         uint4 v = make_uint4(0, 0, 0, 0);
         if (n < G)
           v = __ldg(reinterpret_cast<const uint4*>(
-              p.q + ((size_t)b * p.Hq + h * G + n) * kHeadDim + half * 64 + w16 * 8));
+              p.q + ((size_t)row0 * p.Hq + h * G + n) * kHeadDim + half * 64 + w16 * 8));
         *reinterpret_cast<uint4*>(smem + FC::oQ + half * (N * 128) + n * 128 + ((w16 ^ (n & 7)) << 4)) = v;
       }
       // E4M3 Q: warp w < G splits head row w.  q * 2^e (e puts the row's
@@ -211,7 +219,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
       // 2^-10 x the row maximum).  Rows G..2G-1 hold Q_lo, the rest zero.
       if (sw < G) {
         const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
-            p.q + ((size_t)b * p.Hq + h * G + sw) * kHeadDim + lane * 4));
+            p.q + ((size_t)row0 * p.Hq + h * G + sw) * kHeadDim + lane * 4));
         const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
         const float2 a = __bfloat1622float2(q2[0]), c = __bfloat1622float2(q2[1]);
         float mx = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(c.x), fabsf(c.y)));
@@ -257,7 +265,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   // ------------------------------------------------------------- producer
   if (warp == 0) {
     const uint64_t pol = ptx::l2_policy_evict_first();
-    const int* bt_row = p.block_table + (size_t)b * p.max_pages;
+    const int* bt_row = p.block_table + (size_t)b_seq * p.max_pages;
     auto bt_load = [&](int grp) -> int {
       const int pg = g.sp_begin + 32 * grp + lane;
       return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
@@ -313,7 +321,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   // the tile's bytes take to arrive.
   else if (warp == FC::kVWarp) {
     const uint64_t pol = ptx::l2_policy_evict_first();
-    const int* bt_row = p.block_table + (size_t)b * p.max_pages;
+    const int* bt_row = p.block_table + (size_t)b_seq * p.max_pages;
     auto bt_load = [&](int grp) -> int {
       const int pg = g.sp_begin + 32 * grp + lane;
       return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
@@ -654,7 +662,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
         float o = eo[n * kHeadDim + dd] * sc0 + eo[(RG + n) * kHeadDim + dd] * sc1;
         o = (l > 0.f) ? o * vsc / l : 0.f;
         const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int row = b * p.Hq + h * G + n;
+        const int row = row0 * p.Hq + h * G + n;
         if (p.num_splits == 1) {
           if (p.out_fp32) reinterpret_cast<float*>(p.out)[(size_t)row * kHeadDim + dd] = o;
           else reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * kHeadDim + dd] = __float2bfloat16_rn(o);
@@ -690,7 +698,7 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
     if (bad_cta) atomicOr(p.status, kStatusBadSeq);
   }
   if (aborted_cta || bad_cta)
-    fill_rows<G>(p, first_token_row(p, b), h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    fill_rows<G>(p, row0, h, s_idx, __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, FC::kTmemCols);

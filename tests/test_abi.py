@@ -132,12 +132,24 @@ def test_supported_group_shapes(ra, kw):
     assert ra.rel_attn_workspace_bytes(s, 3) == 256 + (3 * rows * 4 + 255) // 256 * 256 + 3 * rows * 128 * 4
 
 
-def test_e4m3_only_for_one_token(ra):
-    s = shape(ra, num_q_heads=64, num_kv_heads=8, q_tokens=2)
+@pytest.mark.parametrize("kw", [dict(num_q_heads=40, num_kv_heads=8, q_tokens=1),   # G = 5
+                                dict(num_q_heads=64, num_kv_heads=8, q_tokens=9),   # 72 rows
+                                dict(num_q_heads=48, num_kv_heads=8, q_tokens=10)])
+def test_e4m3_rejects_unsupported_shapes(ra, kw):
+    s = shape(ra, **kw)
     fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
     rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
                                      fake, 0, 1, fake, None, fake, 1 << 30, None)
     assert rc == ra.REL_ATTN_ERR_INVALID_ARG
+
+
+def test_e4m3_needs_both_scales(ra):
+    s = shape(ra, num_q_heads=48, num_kv_heads=8, q_tokens=8)
+    fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+    for ks, vs in ((None, fake), (fake, None)):
+        rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(s), fake, fake, fake, ks, vs, fake, fake,
+                                         fake, 0, 1, fake, None, fake, 1 << 30, None)
+        assert rc == ra.REL_ATTN_ERR_INVALID_ARG
 
 
 def test_invalid_pointers_and_splits(ra):

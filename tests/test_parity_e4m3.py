@@ -61,9 +61,9 @@ def check(out, lse, ref_out, ref_lse):
     assert eo <= OUT_TOL and el <= LSE_TOL, (eo, el)
 
 
-def small(L, window=0, NB=1280, seed=0, Hkv=2, lens=None, G=6, **kw):
+def small(L, window=0, NB=1280, seed=0, Hkv=2, lens=None, G=6, T=1, **kw):
     lens = lens if lens is not None else [L]
-    return W.make_case(seq_lens=lens, q_tokens=1, num_q_heads=G * Hkv, num_kv_heads=Hkv,
+    return W.make_case(seq_lens=lens, q_tokens=T, num_q_heads=G * Hkv, num_kv_heads=Hkv,
                        window=window, num_buckets=NB, seed=seed, extra_pages=2, **kw).to("cuda")
 
 
@@ -234,13 +234,67 @@ def test_injected_wait_limit_times_out_cleanly(ra):
     assert ws.read_status() == ra.REL_ATTN_OK
 
 
-def test_rejects_several_query_tokens_and_missing_scales(ra):
-    case = W.make_case(seq_lens=[300], q_tokens=2, num_q_heads=12, num_kv_heads=2,
-                       seed=0).to("cuda")
-    kc, vc, ks, vs = e4m3(case)
-    with pytest.raises(ra.RelAttnError) as e:
-        run_gpu(ra, case, (kc, vc, ks, vs), 1)
-    assert e.value.code == ra.REL_ATTN_ERR_INVALID_ARG
+MULTI = [
+    dict(T=2, L=2), dict(T=2, L=129), dict(T=2, L=3001),
+    dict(T=5, L=5), dict(T=5, L=700, window=64),
+    dict(T=8, L=8), dict(T=8, L=130), dict(T=8, L=4000, seed=2), dict(T=8, L=2500, window=1024),
+    dict(T=9, L=9), dict(T=9, L=3001),
+    dict(T=9, L=1700, G=4, window=512, NB=1024), dict(T=6, L=2100, G=4),
+    dict(T=8, L=3001, G=8), dict(T=3, L=129, G=8),
+    dict(T=4, L=6000, NB=364, exact_buckets=64, max_distance=5000),
+]
+
+
+@pytest.mark.parametrize("kw", MULTI, ids=[str(k) for k in MULTI])
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_several_query_tokens(ra, kw, splits):
+    """A verify step over the E4M3 cache: token t of T sees the keys up to
+    position L - T + t (one-token chunks of the same launch)."""
+    case = small(**kw)
+    codes = e4m3(case)
+    out, lse = run_gpu(ra, case, codes, splits)
+    ref_out, ref_lse = run_oracle(case, codes)
+    check(out, lse, ref_out, ref_lse)
+
+
+def test_several_query_tokens_batched(ra):
+    case = small(0, lens=[9, 130, 2049, 700], T=3, seed=4)
+    codes = e4m3(case)
+    out, lse = run_gpu(ra, case, codes, 0)
+    ref_out, ref_lse = run_oracle(case, codes)
+    check(out, lse, ref_out, ref_lse)
+
+
+def test_verify_256k_eight_tokens_one_kv_head(ra):
+    """The verify shape at full length (262,144 keys, 8 tokens) on one KV
+    head: the oracle computes all 6 x 8 rows."""
+    case = small(262_144, T=8, Hkv=1, seed=7)
+    codes = e4m3(case)
+    out, lse = run_gpu(ra, case, codes, 0)
+    ref_out, ref_lse = run_oracle(case, codes)
+    check(out, lse, ref_out, ref_lse)
+
+
+def test_several_query_tokens_match_one_token_calls(ra):
+    """Token t of a T-token call equals a one-token call whose sequence ends
+    at that token (same splits: the same chunks, bit for bit)."""
+    T, L = 4, 3001
+    case = small(L, T=T, seed=9)
+    codes = e4m3(case)
+    out, lse = run_gpu(ra, case, codes, 3)
+    for t in range(T):
+        one = W.make_case(seq_lens=[L - T + t + 1], q_tokens=1, num_q_heads=12, num_kv_heads=2,
+                          num_buckets=1280, seed=9, extra_pages=2).to("cuda")
+        one.q.copy_(case.q[:, t:t + 1])
+        one.block_table.copy_(case.block_table[:, :one.block_table.shape[1]])
+        kc, vc, ks, vs = codes
+        o1, l1 = ra.rel_attn_decode_e4m3(one.q, kc, vc, ks, vs, one.block_table, one.seq_lens,
+                                         case.rel_table, 0, 3, max_seq_len=L, out_fp32=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o1[:, 0], out[:, t]) and torch.equal(l1[:, 0], lse[:, t]), t
+
+
+def test_rejects_missing_scales(ra):
     import ctypes
     one = small(300)
     kc, vc, ks, vs = e4m3(one)

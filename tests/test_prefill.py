@@ -53,6 +53,9 @@ CASES = [
     dict(C=513, lens=[513]), dict(C=300, lens=[300], window=64),
     dict(C=200, lens=[3000], window=1024, NB=1024), dict(C=64, lens=[64, 200, 1111]),
     dict(C=33, lens=[40, 5000], G=8), dict(C=45, lens=[45, 777], G=4),
+    # nine tokens at G = 8 (72 query rows, the MTP verify the decode instances
+    # do not cover): an 8-token and a 1-token chunk
+    dict(C=9, lens=[9, 2100, 20000], G=8),
     dict(C=24, lens=[1500], NB=364, exact_buckets=64, max_distance=5000),
 ]
 
