@@ -534,37 +534,47 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
-  // Barriers first; the producer starts loading right after, while the other
-  // warps allocate tensor memory and stage Q and the bucket edges.
-  if (tid == 0) {
-    for (int s = 0; s < KS; ++s) {
-      ptx::mbar_init(kfull(s), 1);
-      ptx::mbar_init(kempty(s), 1);
+  // Barriers first, one per lane of warp 0 (in index order: the rings' full /
+  // empty pairs, s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2],
+  // x_full[X], x_empty[X], the two drains; arrival counts 1, or one per
+  // consumer thread for the barriers the softmax threads arrive on).  The
+  // producer's first block-table entries are requested before the CTA-wide
+  // barrier; the other warps then allocate tensor memory and stage Q and the
+  // bucket edges.
+  static_assert(KC::kNumBars <= 32, "one barrier per lane");
+  if (warp == 0) {
+    if (lane < KC::kNumBars) {
+      const int r = lane - kB;
+      const uint32_t cnt =
+          (r < 0) ? 1u
+          : (r < 2) ? 1u                                      // s_full
+          : (r < 6) ? (uint32_t)KC::kConsumers                // s_empty, p_full
+          : (r < 8) ? 1u                                      // o_full
+          : (r < 10) ? (uint32_t)KC::kConsumers               // o_empty
+          : (r < 10 + KC::kXTables) ? 1u                      // x_full
+          : (r < 10 + 2 * KC::kXTables) ? (uint32_t)KC::kConsumers   // x_empty
+          : 1u;                                               // drains
+      ptx::mbar_init(bar0 + 8u * lane, cnt);
+      ptx::fence_mbar_init();
     }
-    for (int s = 0; s < VS; ++s) {
-      ptx::mbar_init(vfull(s), 1);
-      ptx::mbar_init(vempty(s), 1);
+    if (lane == 0) {
+      *abort_flag = 0;
+      *bad_page_flag = 0;
+      issued[0] = issued[1] = 0;
+      ptx::prefetch_tmap(&p.tmap_k);
+      ptx::prefetch_tmap(&p.tmap_v);
+      ptx::prefetch_tmap(&p.tmap_r);
     }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(s_full + 8u * i, 1);
-      ptx::mbar_init(s_empty + 8u * i, KC::kConsumers);
-      ptx::mbar_init(p_full + 8u * i, KC::kConsumers);
-      ptx::mbar_init(o_full + 8u * i, 1);
-      ptx::mbar_init(o_empty + 8u * i, KC::kConsumers);
-    }
-    for (int gq = 0; gq < KC::kXTables; ++gq) {
-      ptx::mbar_init(x_full + 8u * gq, 1);
-      ptx::mbar_init(x_empty + 8u * gq, KC::kConsumers);
-    }
-    ptx::mbar_init(drain_bar, 1);
-    ptx::mbar_init(drain_pv, 1);
-    *abort_flag = 0;
-    *bad_page_flag = 0;
-    issued[0] = issued[1] = 0;
-    ptx::fence_mbar_init();
-    ptx::prefetch_tmap(&p.tmap_k);
-    ptx::prefetch_tmap(&p.tmap_v);
-    ptx::prefetch_tmap(&p.tmap_r);
+  }
+  const int* bt_row = p.block_table + (size_t)b_seq * p.max_pages;
+  auto bt_load = [&](int grp) -> int {
+    const int pg = g.sp_begin + 32 * grp + lane;
+    return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
+  };
+  int bt_cur = 0, bt_next = 0;
+  if (warp == 0) {
+    bt_cur = bt_load(0);
+    bt_next = bt_load(1);
   }
   __syncthreads();
   uint32_t tmem = 0;
@@ -614,13 +624,6 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   // ------------------------------------------------------------- producer
   if (warp == 0) {
     const uint64_t pol = ptx::l2_policy_evict_first();
-    const int* bt_row = p.block_table + (size_t)b_seq * p.max_pages;
-    auto bt_load = [&](int grp) -> int {
-      const int pg = g.sp_begin + 32 * grp + lane;
-      return (pg < g.sp_end) ? __ldg(bt_row + pg) : 0;
-    };
-    int bt_cur = bt_load(0);
-    int bt_next = bt_load(1);
     int k = 0;                                // K-ring items issued
     int i_v = 0;                              // V-ring items (= tiles) issued
     int rows0[2] = {0, 0}, rows1[2] = {0, 0}, npgs[2] = {0, 0};
