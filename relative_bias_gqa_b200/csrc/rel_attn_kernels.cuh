@@ -182,14 +182,21 @@ struct KernelConfig {
   static constexpr int oBar = align_up(oEdges + (kMaxTailBuckets + 1) * 4, 8);
   // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s_full[2],
   //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[kXTables],
-  //           x_empty[kXTables], drain (S issuer), drain (P.V issuer)
-  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 12 + 2 * kXTables;
+  //           x_empty[kXTables], drain (S issuer), drain (P.V issuer),
+  //           plan_full[kPlanSlots], plan_empty[kPlanSlots]
+  // Tile plans (column-split instances): the producer, which plans every
+  // tile for its own loads, hands each plan to the softmax groups through a
+  // ring of kPlanSlots records instead of every softmax thread re-planning.
+  static constexpr int kPlanSlots = kAlt ? 0 : 4;
+  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 12 + 2 * kXTables + 2 * kPlanSlots;
   // tmem base, abort flag, bad-page flag, K-ring and V-ring items issued
   static constexpr int oMisc = oBar + kNumBars * 8;
   // per K slot: 1 if its item is a relative-row chunk, 0 a K tile (producer
   // -> S issuer, published by the slot's full barrier)
   static constexpr int oItemFlag = oMisc + 32;
-  static constexpr int kBytes = oItemFlag + align_up(kKSlots, 16);
+  static constexpr int oPlan = align_up(oItemFlag + kKSlots, 16);   // int4 {k_hi, c0, chunk, 0}
+  static constexpr int kBytes = oPlan + 16 * kPlanSlots;
+  static_assert(oPlan % 16 == 0, "16-byte plan records");
   static constexpr int kAllocBytes = kBytes + 1024;            // 1024-byte alignment slack
   // TMEM columns: S[2] (N each), O[2] (2N each: the P_hi and P_lo halves),
   // per group X0 (and X1 for 136-row chunks)
@@ -524,7 +531,10 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t x_empty = bar0 + 8u * (kB + 10 + KC::kXTables);
   const uint32_t drain_bar = bar0 + 8u * (kB + 10 + 2 * KC::kXTables);
   const uint32_t drain_pv = drain_bar + 8u;
+  auto plan_full = [&](int s) { return drain_pv + 8u * (1 + s); };
+  auto plan_empty = [&](int s) { return drain_pv + 8u * (1 + KC::kPlanSlots + s); };
   uint8_t* item_flag = smem + KC::oItemFlag;
+  int4* plan_rec = reinterpret_cast<int4*>(smem + KC::oPlan);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 4);
   volatile int* bad_page_flag = reinterpret_cast<volatile int*>(smem + KC::oMisc + 8);
@@ -536,7 +546,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   // -------------------------------------------------------------- prologue
   // Barriers first, one per lane of warp 0 (in index order: the rings' full /
   // empty pairs, s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2],
-  // x_full[X], x_empty[X], the two drains; arrival counts 1, or one per
+  // x_full[X], x_empty[X], the two drains, plan_full / plan_empty[kPlanSlots];
+  // arrival counts 1, or one per
   // consumer thread for the barriers the softmax threads arrive on).  The
   // producer's first block-table entries are requested before the CTA-wide
   // barrier; the other warps then allocate tensor memory and stage Q and the
@@ -553,7 +564,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           : (r < 10) ? (uint32_t)KC::kConsumers               // o_empty
           : (r < 10 + KC::kXTables) ? 1u                      // x_full
           : (r < 10 + 2 * KC::kXTables) ? (uint32_t)KC::kConsumers   // x_empty
-          : 1u;                                               // drains
+          : (r < 12 + 2 * KC::kXTables + KC::kPlanSlots) ? 1u        // drains, plan_full
+          : (uint32_t)KC::kConsumers;                         // plan_empty
       ptx::mbar_init(bar0 + 8u * lane, cnt);
       ptx::fence_mbar_init();
     }
@@ -640,6 +652,16 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         const bool odd = KC::kAlt && (ti & 1);
         const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, p.edges, odd ? ps1 : ps0);
         const int c0 = odd ? ps1.c0 : ps0.c0;
+        if constexpr (KC::kPlanSlots > 0) {
+          constexpr int PS = KC::kPlanSlots;
+          ok = __all_sync(0xffffffffu,
+                          ptx::mbar_wait(plan_empty(ti % PS), ((ti / PS) & 1) ^ 1, abort_flag, tlim));
+          if (!ok) break;
+          if (lane == 0) {
+            plan_rec[ti % PS] = make_int4(tp.k_hi, c0, tp.chunk ? 1 : 0, 0);
+            ptx::mbar_arrive(plan_full(ti % PS));
+          }
+        }
         if (tp.chunk) {
           ok = __all_sync(0xffffffffu,
                           ptx::mbar_wait(kempty(k % KS), ((k / KS) & 1) ^ 1, abort_flag, tlim));
@@ -973,9 +995,20 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     for (int ti = t_first; ti < g.ntiles; ti += kStep) {
       TilePlan tp = tp_next;
       int c0 = c0_next;
-      if constexpr (!KC::kAlt) {
-        tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
-        c0 = ps.c0;
+      if constexpr (KC::kPlanSlots > 0) {
+        // the producer's plan of this tile (all threads of the group agree on
+        // whether it arrived before any of them acts on it)
+        constexpr int PS = KC::kPlanSlots;
+        const bool okp = ptx::mbar_wait(plan_full(ti % PS), (ti / PS) & 1, abort_flag, tlim);
+        const int4 rec = okp ? plan_rec[ti % PS] : make_int4(0, 0, 0, 0);
+        ptx::mbar_arrive(plan_empty(ti % PS));
+        if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okp || failed)) { aborted = true; break; }
+        const int pg = g.sp_begin + 2 * ti;
+        tp.j0 = pg * kPage;
+        tp.npg = min(2, g.sp_end - pg);
+        tp.k_hi = rec.x;
+        tp.chunk = rec.z != 0;
+        c0 = rec.y;
       }
       if (tp.chunk) {
         {
