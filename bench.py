@@ -373,6 +373,26 @@ def run_ours(args, rank, world, local_rank):
         eve[i][1].record(stream)
     torch.cuda.synchronize()
     t_e2e = [e[0].elapsed_time(e[1]) for e in eve]
+    # Breakdown of the same step with the device held by a short sleep while
+    # the host queues it (as in the main loop), events between the parts:
+    # copy in, call, copy out; the rest of the end-to-end time is the device
+    # waiting for the host to submit the next part.
+    Kb = min(K, 500)
+    evb = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(Kb)]
+    for i in range(Kb):
+        flush.zero_()
+        torch.cuda._sleep(sleep_cycles)
+        evb[i][0].record(stream)
+        d_in.copy_(h_in, non_blocking=True)
+        evb[i][1].record(stream)
+        prep_e2e.decode()
+        evb[i][2].record(stream)
+        h_res.copy_(d_res, non_blocking=True)
+        evb[i][3].record(stream)
+    torch.cuda.synchronize()
+    t_in = statistics.fmean(e[0].elapsed_time(e[1]) for e in evb) * 1e3
+    t_call = statistics.fmean(e[1].elapsed_time(e[2]) for e in evb) * 1e3
+    t_out = statistics.fmean(e[2].elapsed_time(e[3]) for e in evb) * 1e3
     prep.decode()
     torch.cuda.synchronize()
     if not (torch.equal(prep.out, d_out) and torch.equal(prep.lse, d_lse)):
@@ -453,9 +473,17 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "us_per_call": round(statistics.fmean(t_e2e) * 1e3, 2),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "breakdown_us": {"copy_in": round(t_in, 2), "call": round(t_call, 2),
+                                     "copy_out": round(t_out, 2),
+                                     "rest": round(statistics.fmean(t_e2e) * 1e3
+                                                   - t_in - t_call - t_out, 2)},
                     "note": "q, block table and seq_lens copied in from one pinned host buffer and "
                             "out + lse copied back into one inside each timed step (one copy "
-                            "each way); the KV cache and relative table are resident model state"},
+                            "each way); the KV cache and relative table are resident model state. "
+                            "breakdown_us: the same step queued ahead behind a device sleep, "
+                            "events between its parts (each event pair adds about 2 us); rest = "
+                            "us_per_call minus the three parts: host submission gaps less the "
+                            "extra events' cost"},
             "gpu_launches": K * (2 if S > 1 else 1),
             "timed_region": "K rel_attn_decode calls (partial kernel + PDL-chained combine kernel); "
                             "us_partial_kernel from a second loop with an event between the kernels",
