@@ -13,6 +13,13 @@
  * bucket(d): d for d < E (E = exact_buckets, 1024); beyond that NL = NB - E
  * log-spaced buckets with lower edges e_k = ceil(E (Dmax/E)^(k/NL)),
  * bucket = E + min(NL-1, max{k : e_k <= d}); when NB <= E, min(d, NB-1).
+ * The kernels read the relative rows a 128-key tile needs as one contiguous
+ * block of 128 rows (one query token per kernel) or 136 (several), so any
+ * 127 + T consecutive distances must span at most that many bucket indices.
+ * The standard table (NB 1,280, E 1,024, Dmax 2^20) spans 128 / 129..136;
+ * a table whose tail buckets start narrower than one distance can span more
+ * and is refused by the compute entry points with REL_ATTN_ERR_INVALID_ARG
+ * (rel_attn_bucket still evaluates it).
  *
  * Sources: "vLLM TML Inkling 지원", section "TML Inkling 모델 아키텍처"
  * (learned relative term added to the pre-softmax logits instead of RoPE;

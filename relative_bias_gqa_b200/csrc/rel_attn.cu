@@ -161,6 +161,9 @@ struct EdgeEntry {
   int nb = -1, e = -1, dmax = -1, ex = 0, nl = 0;
   float log2_ex = 0.f, log_scale = 0.f;
   int edges[kMaxTailBuckets + 1];
+  // largest number of bucket indices that 127 + T consecutive distances
+  // span (index T = 1..kMaxQTokens), see bucket_span_fits
+  int max_span[kMaxQTokens + 1];
 };
 struct MapEntry { const void* base = nullptr; uint64_t a = 0, b = 0; int kind = -1; CUtensorMap map; };
 constexpr int kEdgeCache = 4, kMapCache = 16;
@@ -168,6 +171,26 @@ EdgeEntry g_edge_cache[kEdgeCache];
 MapEntry g_map_cache[kMapCache];
 int g_edge_next = 0, g_map_next = 0;
 std::mutex g_cache_mu;
+
+int bucket_host(int d, int ex, int nl, const int* edges);
+
+// Bucket indices spanned by the distances [d, d + W - 1], maximised over d.
+// bucket() is non-decreasing, so the maximum is taken at a distance where a
+// bucket starts: every exact distance and every tail edge.
+void fill_max_spans(EdgeEntry& e) {
+  for (int T = 1; T <= kMaxQTokens; ++T) {
+    const long long W = 127 + T;
+    int best = 0;
+    auto span_at = [&](long long d) {
+      const long long d1 = std::min<long long>(d + W - 1, INT32_MAX);
+      const int sp = bucket_host((int)d1, e.ex, e.nl, e.edges) - bucket_host((int)d, e.ex, e.nl, e.edges) + 1;
+      best = std::max(best, sp);
+    };
+    for (int d = 0; d <= e.ex; ++d) span_at(d);
+    for (int k = 0; k <= e.nl && e.nl > 0; ++k) span_at(e.edges[k]);
+    e.max_span[T] = best;
+  }
+}
 
 void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges,
                          float* log2_ex = nullptr, float* log_scale = nullptr) {
@@ -183,6 +206,7 @@ void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges,
     EdgeEntry& e = g_edge_cache[g_edge_next++ % kEdgeCache];
     bucket_table(s, &e.ex, &e.nl, e.edges, &e.log2_ex, &e.log_scale);
     e.nb = s->num_buckets; e.e = s->exact_buckets; e.dmax = s->max_distance;
+    fill_max_spans(e);
     hit = &e;
   }
   *ex = hit->ex;
@@ -190,6 +214,28 @@ void bucket_table_cached(const rel_attn_shape* s, int* ex, int* nl, int* edges,
   if (log2_ex) *log2_ex = hit->log2_ex;
   if (log_scale) *log_scale = hit->log_scale;
   memcpy(edges, hit->edges, sizeof(int) * (hit->nl + 1));
+}
+
+// Whether one relative-row chunk holds every bucket a tile can need: the
+// 127 + T distances of a 128-key tile (T query tokens) must span at most
+// 128 bucket indices for one token and 136 for several (the chunk's rows).
+// A table whose tail buckets are narrower than a distance near the exact
+// range can span more; such tables are rejected.  kernel_tokens is the T the
+// partial kernel runs with (1 for the E4M3 kernel, whose tokens are chunks).
+bool bucket_span_fits(const rel_attn_shape* s, int kernel_tokens) {
+  int ex, nl;
+  static thread_local int edges[kMaxTailBuckets + 1];
+  bucket_table_cached(s, &ex, &nl, edges);
+  int span = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    for (auto& e : g_edge_cache)
+      if (e.nb == s->num_buckets && e.e == s->exact_buckets && e.dmax == s->max_distance) {
+        span = e.max_span[kernel_tokens];
+        break;
+      }
+  }
+  return span >= 1 && span <= (kernel_tokens == 1 ? 128 : 136);
 }
 
 int bucket_host(int d, int ex, int nl, const int* edges) {
@@ -458,6 +504,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   // ---- validation (no CUDA call before this block passes)
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
+  if (!bucket_span_fits(shape, kv_e4m3 ? 1 : shape->q_tokens)) return REL_ATTN_ERR_INVALID_ARG;
   if (kv_e4m3) {
     if (!k_scale || !v_scale ||
         (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))

@@ -961,19 +961,28 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 
     // Accumulate the O^T tile of tile j (this thread's head-dim lane, this
     // group's columns) with the rescale factors `al` of that tile.
-    auto process_o = [&](int j, const float* al) {
+    // `rescaled` false: the tile kept every reference max (alpha = 1), and
+    // the factors are not read.
+    auto process_o = [&](int j, const float* al, bool rescaled) {
       float ov[RG8 * 8];
       const bool okw = ptx::mbar_wait(o_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim);
       if (okw) {
         ptx::tc_fence_after();
         const uint32_t ob = tO + lane_off + (j & 1) * 2 * N;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {          // O^T from P_hi, then from P_lo
-          ld_rows(ob + part * N, ov);
+        ld_rows(ob, ov);                                 // O^T from P_hi
+        if (rescaled) {
 #pragma unroll
           for (int r = 0; r < RG; ++r)
-            if (live(r)) o_acc[r] = part ? o_acc[r] + ov[r] : fmaf(o_acc[r], al[r], ov[r]);
+            if (live(r)) o_acc[r] = fmaf(o_acc[r], al[r], ov[r]);
+        } else {
+#pragma unroll
+          for (int r = 0; r < RG; ++r)
+            if (live(r)) o_acc[r] += ov[r];
         }
+        ld_rows(ob + N, ov);                             // then from P_lo
+#pragma unroll
+        for (int r = 0; r < RG; ++r)
+          if (live(r)) o_acc[r] += ov[r];
         ptx::tc_fence_before();
       }
       ptx::mbar_arrive(o_empty + 8u * (j & 1));
@@ -981,6 +990,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     };
 
     int last_tile = -1;
+    bool resc_prev = false;                   // tile last_tile moved some reference max
     // This group's tiles: every other one (alternating groups) or all.  With
     // alternating groups the plan of the group's next tile is made while P.V
     // of the current one runs (elsewhere the registers are scarcer).
@@ -1089,7 +1099,9 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       for (int r = 0; r < RG; ++r)
         if (live(r)) over |= s[r] > m_ref[r] + kLazyLog2;
       float* al_buf = alpha_buf + (li & 1) * KC::kGR;
+      bool resc_now = false;                  // this tile moved some reference max
       if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, over || !okw || failed)) {
+        resc_now = true;
         if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, !okw || failed)) { aborted = true; break; }
         float* redb = red + (li & 1) * 4 * KC::kGR;
 #pragma unroll
@@ -1113,12 +1125,9 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             m_ref[r] = mn;
           }
         }
-      } else {
+      } else if constexpr (KC::kAlt) {
 #pragma unroll
-        for (int r = 0; r < RG; ++r) {
-          if constexpr (KC::kAlt) alpha_r[r] = 1.f;
-          else if (kl == 0 && live(r)) al_buf[r] = 1.f;
-        }
+        for (int r = 0; r < RG; ++r) alpha_r[r] = 1.f;
       }
       // ---- P = exp2(x - m_ref) as bf16 hi + lo parts (~16 significant bits in
       //      the P.V product), stacked [P_hi; P_lo] = 2N rows, MN-major without
@@ -1131,7 +1140,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if constexpr (KC::kPBufs == 1) {
         // one P buffer: P.V(i-1) must have read it before P(i) goes in, and
         // taking O(i-1) waits for exactly that
-        if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
+        if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR, resc_prev);
       }
       {
         constexpr int U = kAlign;                              // rows per store
@@ -1199,20 +1208,21 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       }
       if constexpr (KC::kAlt) {
         // this group's next tile is i + 2: take O(i) now
-        process_o(i, alpha_r);
+        process_o(i, alpha_r, true);
       } else if constexpr (KC::kPBufs == 2) {
         // every group is on every tile: take O(i-1) while P.V(i) runs
         if (last_tile >= 0) {
-          process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
+          process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR, resc_prev);
         }
       }
+      resc_prev = resc_now;
       last_tile = i;
       ++li;
     }
     if constexpr (!KC::kAlt) {
       if (!aborted) {
         if (ptx::bar_sync_or(bar_id, kSoftmaxThreads, failed)) aborted = true;
-        else if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR);
+        else if (last_tile >= 0) process_o(last_tile, alpha_buf + ((li - 1) & 1) * KC::kGR, resc_prev);
       }
     }
     ptx::pdl_launch_dependents();

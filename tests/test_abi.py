@@ -259,3 +259,42 @@ def test_e4m3_partition_gives_the_exact_range_fewer_pages(ra):
     a8, b8 = ra.rel_attn_split_pages(s, L, 0, 18, 17, e4m3=True)
     assert b16 == b8 == (L - 1) // 64 + 1
     assert b8 - a8 < b16 - a16
+
+
+def _span_oracle(nb, e, dmax, T):
+    """Largest number of bucket indices that 127 + T consecutive distances
+    span, from the oracle's bucket function (bucket() is non-decreasing, so
+    windows starting where a bucket starts suffice)."""
+    import oracle
+    edges = oracle.log_bucket_edges(nb, e, dmax) if nb > e else np.array([], dtype=np.int64)
+    starts = np.unique(np.concatenate([np.arange(0, e + 1), edges])).astype(np.int64)
+    starts = starts[starts < (1 << 31) - 200]
+    b0 = oracle.bucket_of_distance(starts, nb, e, dmax)
+    b1 = oracle.bucket_of_distance(starts + 126 + T, nb, e, dmax)
+    return int((b1 - b0 + 1).max())
+
+
+@pytest.mark.parametrize("nb,e,dmax", EDGE_TRIPLES + [(600, 100, 8000), (350, 100, 1500)],
+                         ids=[str(t) for t in EDGE_TRIPLES + [(600, 100, 8000), (350, 100, 1500)]])
+@pytest.mark.parametrize("T", [1, 2, 8])
+def test_bucket_tables_too_dense_for_a_chunk_are_rejected(ra, nb, e, dmax, T):
+    """A tile's 127 + T distances must span at most 128 bucket indices for
+    one token (136 for several): one relative-row chunk then holds every
+    bucket the tile needs.  Denser tables are refused before any CUDA call;
+    the others pass validation (and fail later only for the fake pointers,
+    with NO_DEVICE on a machine without a GPU)."""
+    s = shape(ra, num_buckets=nb, exact_buckets=e, max_distance=dmax, q_tokens=T,
+              num_q_heads=48, num_kv_heads=8)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = ra.lib.rel_attn_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 0, 1, fake,
+                                None, fake, 1 << 30, None)
+    too_dense = _span_oracle(nb, e, dmax, T) > (128 if T == 1 else 136)
+    if too_dense:
+        assert rc == ra.REL_ATTN_ERR_INVALID_ARG
+    elif not torch.cuda.is_available():
+        assert rc == ra.REL_ATTN_ERR_NO_DEVICE
+
+
+def test_dense_table_in_the_edge_tests_is_too_dense(ra):
+    assert _span_oracle(600, 100, 1500, 1) > 128 and _span_oracle(600, 100, 1500, 2) > 136
+    assert _span_oracle(1280, 1024, 1 << 20, 1) == 128 and _span_oracle(1280, 1024, 1 << 20, 8) == 135

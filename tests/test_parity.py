@@ -77,7 +77,10 @@ SMALL = [
     # edges, and distances past max_distance clamped into the last bucket
     dict(L=6000, NB=364, exact_buckets=64, max_distance=5000),
     dict(L=3000, T=8, NB=200, exact_buckets=16, max_distance=100000),
-    dict(L=2200, T=2, NB=600, exact_buckets=100, max_distance=1500),
+    # dense tail buckets (nearly one per distance past the exact range): the
+    # densest tables one relative-row chunk still covers
+    dict(L=2200, T=2, NB=600, exact_buckets=100, max_distance=8000),
+    dict(L=3000, T=8, NB=350, exact_buckets=100, max_distance=1500),
 ]
 
 
