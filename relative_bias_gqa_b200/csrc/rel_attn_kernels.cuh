@@ -1023,7 +1023,8 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       if (tp.chunk) {
         {
           // ---- new relative-row chunk: this group's columns of X^T (128 or
-          //      136 relative rows) -> gather table Y
+          //      136 relative rows) -> gather table Y, already multiplied by
+          //      the logit scale so that each logit is one fma
           const int xb = KC::kAlt ? grp : 0;
           const bool okw = ptx::mbar_wait(x_full + 8u * xb, c & 1, abort_flag, tlim);
           if (okw) {
@@ -1032,13 +1033,13 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
             ld_rows(tXg, xv);
 #pragma unroll
             for (int r = 0; r < RG; ++r)
-              if (live(r)) Y[kl * YS + slot0 + r] = xv[r];
+              if (live(r)) Y[kl * YS + slot0 + r] = xv[r] * p.scale_log2;
             if (ROWS > 128 && sp == 3) {         // rows 128..135 come from lanes 120..127 of X1
               ld_rows(tXg + N, xv);
               if (lane >= 24) {
 #pragma unroll
                 for (int r = 0; r < RG; ++r)
-                  if (live(r)) Y[(kl + 8) * YS + slot0 + r] = xv[r];
+                  if (live(r)) Y[(kl + 8) * YS + slot0 + r] = xv[r] * p.scale_log2;
               }
             }
             ptx::tc_fence_before();
@@ -1086,7 +1087,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
           const int r = tt * G + gg;
-          s[r] = v ? (s[r] + yrow[r]) * p.scale_log2 : -INFINITY;
+          s[r] = v ? fmaf(s[r], p.scale_log2, yrow[r]) : -INFINITY;
         }
       }
       // ---- lazy max: p = exp2(x - m_ref) with the row's reference max
