@@ -319,9 +319,11 @@ int rel_attn_set_wait_limit(unsigned long long limit_ns);
 int rel_attn_read_status(void* workspace, void* stream);
 
 /* The split heuristic: KV splits per (sequence, KV head) so that
- * batch * Hkv * splits fills `sm_count` SMs, bounded by the work available
- * (at least one 128-key tile per split) and by 256.  sm_count <= 0 queries
- * the current device.  Returns >= 1, or a negative error code. */
+ * batch * Hkv * splits fills `sm_count` SMs in one wave when batch * Hkv <
+ * sm_count, and otherwise gives about twelve CTAs per SM in all (short
+ * CTAs even out sequences of different lengths), bounded by the work
+ * available (at least one 128-key tile per split) and by 256.  sm_count <= 0
+ * queries the current device.  Returns >= 1, or a negative error code. */
 int rel_attn_choose_splits(const rel_attn_shape* shape, int window, int sm_count);
 
 /* bucket(distance) exactly as the kernels compute it (host copy of the same

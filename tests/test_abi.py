@@ -172,10 +172,12 @@ def test_split_heuristic_values(ra):
     assert ra.rel_attn_choose_splits(shape(ra), 1024, 148) == 9
     # small contexts: at most one split per 128-key tile
     assert ra.rel_attn_choose_splits(shape(ra, max_seq_len=300), 0, 148) == 3
-    # 32 sequences x 8 heads > 148 SMs: a few splits for load balance
+    # 32 sequences x 8 heads > 148 SMs: about twelve CTAs per SM in all
     s = shape(ra, batch=32, max_seq_len=131_072, max_pages_per_seq=2048, num_pages=40000)
-    v = ra.rel_attn_choose_splits(s, 0, 148)
-    assert 1 <= v <= 4
+    assert ra.rel_attn_choose_splits(s, 0, 148) == 7         # ceil(12 * 148 / 256)
+    # many units: one split each
+    s = shape(ra, batch=2048, max_seq_len=131_072, max_pages_per_seq=2048, num_pages=40000)
+    assert ra.rel_attn_choose_splits(s, 0, 148) == 1
     for sm in (1, 7, 148, 1000):
         assert 1 <= ra.rel_attn_choose_splits(shape(ra), 0, sm) <= 256
     # the previous Inkling's layers: 64/8 full behaves like 48/8 (8 KV heads);
