@@ -4,9 +4,8 @@
 //   warp 0      TMA producer: walks the split's pages through the block table
 //               and streams K/V page tiles (and relative-table row chunks)
 //               into a ring of 64 KB shared-memory stages.
-//   warp 1      MMA issuer (one thread; in most instances it issues S and X
-//               and a warp after the softmax warps issues P.V): tcgen05.mma
-//               with fp32 accumulators
+//   warp 1      S / X issuer, and after the softmax warps a P.V issuer (one
+//               thread each): tcgen05.mma with fp32 accumulators
 //               in tensor memory, "swap-AB" orientation so that keys (and
 //               head-dim for P.V) fill the 128-row M side and the GQA
 //               group's G heads x T tokens are the N side:
@@ -137,15 +136,13 @@ struct KernelConfig {
   // rows.  N = 32 / 48 / 64 (2..9 tokens): every group takes every tile, each
   // with its own block of rows (a column split of S^T, X^T and O^T).
   static constexpr bool kAlt = (N == 16);
-  // warp 0 producer, warp 1 MMA issuer, the softmax warps.  kSplitIssue:
-  // warp 1 issues S and X only and a warp after the softmax warps issues
-  // P.V.  Measured on B200 (256K-key verify step, tokens 1..9): faster with
-  // two groups and with an odd token count over four groups (7 and 9 tokens
-  // at G = 6: 274 -> 267 and 543 -> 510 us), slower with an even one (6 and 8
-  // tokens: 262 -> 271 and 251 -> 260 us).
-  static constexpr bool kSplitIssue = (NG == 2) || (T % 2 == 1);
-  static constexpr int kPvWarp = kSplitIssue ? 2 + 4 * NG : -1;
-  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + (kSplitIssue ? 32 : 0);
+  // warp 0 producer, warp 1 S / X issuer, the softmax warps, then the P.V
+  // issuer.  Measured on B200 against one thread issuing both (256K-key
+  // verify step): 4 tokens 210 -> 189 us, 6 tokens 222 -> 206, 8 tokens 238
+  // -> 237; 100K keys at G = 8 with 8 tokens 146 -> 134; batched_32 1,945 ->
+  // 1,702 (before the split heuristic changed).
+  static constexpr int kPvWarp = 2 + 4 * NG;
+  static constexpr int kThreads = 64 + kSoftmaxThreads * NG + 32;
   static constexpr int kConsumers = kAlt ? kSoftmaxThreads : kSoftmaxThreads * NG;  // arrivals per tile
   static constexpr int kXTables = kAlt ? NG : 1;               // relative chunks in flight (X, Y)
   // row capacity of a group: N / NG, or more when the tokens do not split
@@ -594,7 +591,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     if (warp == 1) {
       ptx::tmem_alloc(ptx::smem_addr(tmem_holder), KC::kTmemCols);
       ptx::tmem_relinquish();
-    } else if (!KC::kSplitIssue || warp != KC::kPvWarp) {
+    } else if (warp != KC::kPvWarp) {
       const int st = tid - 64;
       const int nst = kSoftmaxThreads * NG;
       // Q group tile, 128B-swizzled K-major: query slot n holds (token t,
@@ -725,152 +722,62 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     }
   }
   // ------------------------------------------------------- S and X issuer
-  // With kSplitIssue, S / X and P.V are issued by two warps side by side: one
-  // issuing thread spends most of a microsecond per tile on its waits,
-  // descriptors and MMA issues, close to what the tile's bytes take at the
-  // HBM rate.  Otherwise this thread issues both, P.V of the previous tile
-  // first unless this tile's K data has already landed.
+  // S / X and P.V are issued by two warps side by side: one issuing thread
+  // spends most of a microsecond per tile on its waits, descriptors and MMA
+  // issues, close to what the tile's bytes take at the HBM rate.
   else if (warp == 1) {
     if (lane == 0) {
-      if constexpr (KC::kSplitIssue) {
-        constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
-        // Base descriptors; every MMA operand below is one of these plus a
-        // constant byte offset (the address field is the low 14 bits, >> 4).
-        const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
-        const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
-        int k = 0;                               // K-ring items taken
-        int cg[2] = {0, 0};                      // chunks issued per group
-        for (int ti = 0; ti < g.ntiles; ++ti) {
-          const int gq = KC::kAlt ? (ti & 1) : 0;
-          if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
-          if (item_flag[k % KS]) {
-            // the tile's new relative-row chunk came first: X = R_chunk . Q
-            const int c = cg[gq];
-            if (!ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim)) break;
-            ptx::tc_fence_after();
-            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
-              const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
-              ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
-              if constexpr (ROWS > 128)
-                ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
-            }
-            ptx::umma_commit(x_full + 8u * gq);
-            ptx::umma_commit(kempty(k % KS));
-            ++k;
-            cg[gq] = c + 1;
-            if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
-          }
-          if (!ptx::mbar_wait(s_empty + 8u * (ti & 1), ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
+      constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
+      // Base descriptors; every MMA operand below is one of these plus a
+      // constant byte offset (the address field is the low 14 bits, >> 4).
+      const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
+      const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
+      int k = 0;                               // K-ring items taken
+      int cg[2] = {0, 0};                      // chunks issued per group
+      for (int ti = 0; ti < g.ntiles; ++ti) {
+        const int gq = KC::kAlt ? (ti & 1) : 0;
+        if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
+        if (item_flag[k % KS]) {
+          // the tile's new relative-row chunk came first: X = R_chunk . Q
+          const int c = cg[gq];
+          if (!ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim)) break;
           ptx::tc_fence_after();
           const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            ptx::umma_bf16(tS + (ti & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
-                           qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
+            const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
+            const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+            ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
+            if constexpr (ROWS > 128)
+              ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
           }
-          ptx::umma_commit(s_full + 8u * (ti & 1));
-          ptx::umma_commit(kempty(k % KS));        // the K slot is free once S is done
+          ptx::umma_commit(x_full + 8u * gq);
+          ptx::umma_commit(kempty(k % KS));
           ++k;
+          cg[gq] = c + 1;
+          if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
         }
-        // every MMA issued so far must finish before tensor memory is released
-        ptx::umma_commit(drain_bar);
-        volatile int never = 0;
-        ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
-      } else {
-        constexpr uint32_t kIdescQK = ptx::idesc_bf16(128, N, false, false);
-        constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
-        // Base descriptors; every MMA operand below is one of these plus a
-        // constant byte offset (the address field is the low 14 bits, >> 4).
-        const uint64_t kdesc0 = ptx::sdesc_sw128(sbase + KC::oK, 16, 1024);          // K / R chunk, K-major
-        const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
-        const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + KC::oV, kHalfTileBytes, 1024);  // V^T, MN-major
-        const uint64_t pdesc0 = ptx::sdesc_noswz(sP0, 16 * 2 * N, 128);              // [P_hi; P_lo], MN-major
-        int k = 0, i = 0;                        // K-ring items, tiles issued
-        int cg[2] = {0, 0};                      // chunks issued per group
-        PlanState ps0(p.nl), ps1(p.nl);
-        bool ok = true;
-        auto issue_pv = [&](int j) -> bool {
-          if (!ptx::mbar_wait(p_full + 8u * (j & 1), (j >> 1) & 1, abort_flag, tlim)) return false;
-          if (!ptx::mbar_wait(o_empty + 8u * (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, tlim)) return false;
-          if (!ptx::mbar_wait(vfull(j % VS), (j / VS) & 1, abort_flag, tlim)) return false;
-          ptx::tc_fence_after();
-          const uint64_t va = vdesc0 + (uint64_t)(((j % VS) * kVSlotBytes) >> 4);
-          const uint64_t pbd = pdesc0 + (uint64_t)(((j % KC::kPBufs) * KC::kPBufBytes) >> 4);
-          // B = [P_hi; P_lo] (2N rows): one pass over V gives O^T for both parts
+        if (!ptx::mbar_wait(s_empty + 8u * (ti & 1), ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
+        ptx::tc_fence_after();
+        const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            ptx::umma_bf16(tO + (j & 1) * 2 * N, va + (uint64_t)((kk * 2048) >> 4),
-                           pbd + (uint64_t)((kk * (2 * 16 * 2 * N)) >> 4), kIdescPV, kk > 0);
-          }
-          ptx::umma_commit(o_full + 8u * (j & 1));
-          ptx::umma_commit(vempty(j % VS));
-          return true;
-        };
-        for (int ti = 0; ti < g.ntiles; ++ti) {
-          const int gq = KC::kAlt ? (ti & 1) : 0;
-          const TilePlan tp = plan_tile<ROWS>(g, ti, p.ex, p.log2_ex, p.log_scale, s_edges, gq ? ps1 : ps0);
-          // P.V of the previous tile frees a V slot: issue it first unless this
-          // tile's K data has already landed (then S first, so softmax starts).
-          bool pv_pending = i > 0;
-          if (pv_pending) {
-            const int kt = k + (tp.chunk ? 1 : 0);
-            if (!ptx::mbar_try_wait(kfull(kt % KS), (kt / KS) & 1)) {
-              if (!(ok = issue_pv(i - 1))) break;
-              pv_pending = false;
-            }
-          }
-          if (tp.chunk) {
-            const int c = cg[gq];
-            ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
-                 ptx::mbar_wait(x_empty + 8u * gq, (c & 1) ^ 1, abort_flag, tlim);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t ra = kd + (uint64_t)(((kk >> 2) * KC::kRHalfBytes + (kk & 3) * 32) >> 4);
-              const uint64_t bq = qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
-              ptx::umma_bf16(tX(gq), ra, bq, kIdescQK, kk > 0);
-              if constexpr (ROWS > 128)
-                ptx::umma_bf16(tX(gq) + N, ra + (uint64_t)(1024 >> 4), bq, kIdescQK, kk > 0);
-            }
-            ptx::umma_commit(x_full + 8u * gq);
-            ptx::umma_commit(kempty(k % KS));
-            ++k;
-            cg[gq] = c + 1;
-          }
-          ok = ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim) &&
-               ptx::mbar_wait(s_empty + 8u * (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, tlim);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          {
-            const uint64_t kd = kdesc0 + (uint64_t)(((k % KS) * KC::kKSlotBytes) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              ptx::umma_bf16(tS + (i & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
-                             qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
-            }
-            ptx::umma_commit(s_full + 8u * (i & 1));
-            ptx::umma_commit(kempty(k % KS));      // the K slot is free once S is done
-          }
-          if (pv_pending && !(ok = issue_pv(i - 1))) break;
-          ++k;
-          ++i;
+        for (int kk = 0; kk < 8; ++kk) {
+          ptx::umma_bf16(tS + (ti & 1) * N, kd + (uint64_t)(((kk >> 2) * kHalfTileBytes + (kk & 3) * 32) >> 4),
+                         qdesc0 + (uint64_t)(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
         }
-        if (ok && i > 0) ok = issue_pv(i - 1);
-        // every MMA issued so far must finish before tensor memory is released
-        ptx::umma_commit(drain_bar);
-        volatile int never = 0;
-        ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
+        ptx::umma_commit(s_full + 8u * (ti & 1));
+        ptx::umma_commit(kempty(k % KS));        // the K slot is free once S is done
+        ++k;
       }
+      // every MMA issued so far must finish before tensor memory is released
+      ptx::umma_commit(drain_bar);
+      volatile int never = 0;
+      ptx::mbar_wait(drain_bar, 0, &never, kDrainLimitNs);
     }
     __syncwarp();
   }
   // ----------------------------------------------------------- P.V issuer
-  else if (KC::kSplitIssue && warp == KC::kPvWarp) {
+  else if (warp == KC::kPvWarp) {
     if (lane == 0) {
       constexpr uint32_t kIdescPV = ptx::idesc_bf16(128, 2 * N, true, true);
       const uint64_t vdesc0 = ptx::sdesc_sw128(sbase + KC::oV, kHalfTileBytes, 1024);  // V^T, MN-major
