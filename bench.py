@@ -393,10 +393,40 @@ def run_ours(args, rank, world, local_rank):
     t_in = statistics.fmean(e[0].elapsed_time(e[1]) for e in evb) * 1e3
     t_call = statistics.fmean(e[1].elapsed_time(e[2]) for e in evb) * 1e3
     t_out = statistics.fmean(e[2].elapsed_time(e[3]) for e in evb) * 1e3
+    # The same step with the result written by the kernels straight into a
+    # pinned host buffer (mapped host memory: under unified addressing its
+    # host address is valid on the device), instead of a device-to-host copy
+    # after the call; taken only when the runtime confirms the mapping.
+    h_zc, (h_out_zc, h_lse_zc) = packed(out_parts, "pin")
+    try:
+        try:
+            from cuda.bindings import runtime as cudart
+        except ImportError:
+            from cuda import cudart
+        err, dptr = cudart.cudaHostGetDevicePointer(h_zc.data_ptr(), 0)
+        mapped = int(err) == 0 and int(dptr) == h_zc.data_ptr()
+    except Exception:
+        mapped = False
+    t_zc = None
+    if mapped:
+        prep_zc = rel_attn.Prepared(d_q, kv_args["k_cache"], kv_args["v_cache"], d_bt, d_sl,
+                                    case.rel_table, case.window, S, out=h_out_zc, lse=h_lse_zc,
+                                    max_seq_len=case.max_seq_len, out_fp32=False, **kv_args["scales"])
+        evz = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+        for i in range(Ke):
+            flush.zero_()
+            evz[i][0].record(stream)
+            d_in.copy_(h_in, non_blocking=True)
+            prep_zc.decode()
+            evz[i][1].record(stream)
+        torch.cuda.synchronize()
+        t_zc = [e[0].elapsed_time(e[1]) for e in evz]
     prep.decode()
     torch.cuda.synchronize()
     if not (torch.equal(prep.out, d_out) and torch.equal(prep.lse, d_lse)):
         raise RuntimeError("packed end-to-end call disagrees with the resident-input call")
+    if mapped and not (torch.equal(prep.out.cpu(), h_out_zc) and torch.equal(prep.lse.cpu(), h_lse_zc)):
+        raise RuntimeError("zero-copy end-to-end call disagrees with the resident-input call")
     h2d = h_in.numel()
     d2h = h_res.numel()
 
@@ -435,7 +465,8 @@ def run_ours(args, rank, world, local_rank):
         achieved = nbytes / (kernel_ms * 1e-3) / 1e9
         value = whole_job_gbs(world, K, nbytes, total_ms)
         src_hash = kernel_source_hash()
-        e2e_gbs = world * nbytes / (statistics.fmean(t_e2e) * 1e-3) / 1e9
+        t_best = t_zc if (t_zc is not None and statistics.fmean(t_zc) < statistics.fmean(t_e2e)) else t_e2e
+        e2e_gbs = world * nbytes / (statistics.fmean(t_best) * 1e-3) / 1e9
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -471,19 +502,26 @@ def run_ours(args, rank, world, local_rank):
                                  "whole layer-call (partial + combine) per GPU"},
             "parity": parity,
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
-                    "us_per_call": round(statistics.fmean(t_e2e) * 1e3, 2),
+                    "us_per_call": round(statistics.fmean(t_best) * 1e3, 2),
+                    "result_to_host": "kernel stores into mapped pinned memory" if t_best is t_zc
+                                      else "one device-to-host copy",
+                    "us_per_call_copy_out": round(statistics.fmean(t_e2e) * 1e3, 2),
+                    "us_per_call_zero_copy_out": (round(statistics.fmean(t_zc) * 1e3, 2)
+                                                  if t_zc is not None else None),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "breakdown_us": {"copy_in": round(t_in, 2), "call": round(t_call, 2),
                                      "copy_out": round(t_out, 2),
                                      "rest": round(statistics.fmean(t_e2e) * 1e3
                                                    - t_in - t_call - t_out, 2)},
-                    "note": "q, block table and seq_lens copied in from one pinned host buffer and "
-                            "out + lse copied back into one inside each timed step (one copy "
-                            "each way); the KV cache and relative table are resident model state. "
-                            "breakdown_us: the same step queued ahead behind a device sleep, "
-                            "events between its parts (each event pair adds about 2 us); rest = "
-                            "us_per_call minus the three parts: host submission gaps less the "
-                            "extra events' cost"},
+                    "note": "q, block table and seq_lens copied in from one pinned host buffer "
+                            "inside each timed step; out + lse reach pinned host memory either by "
+                            "one copy after the call (us_per_call_copy_out) or written there by "
+                            "the kernels themselves (mapped memory, us_per_call_zero_copy_out); "
+                            "us_per_call is the faster. The KV cache and relative table are "
+                            "resident model state. breakdown_us (copy-out form): the same step "
+                            "queued ahead behind a device sleep, events between its parts (each "
+                            "event pair adds about 2 us); rest = us_per_call_copy_out minus the "
+                            "three parts"},
             "gpu_launches": K * (2 if S > 1 else 1),
             "timed_region": "K rel_attn_decode calls (partial kernel + PDL-chained combine kernel); "
                             "us_partial_kernel from a second loop with an event between the kernels",
