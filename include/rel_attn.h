@@ -36,17 +36,21 @@
  * Conventions for every entry point:
  *   - Tensor arguments are DEVICE pointers owned by the caller; the library
  *     never allocates, frees or retains them.  Host-side arguments are the
- *     shape struct and scalars.
+ *     shape struct and scalars.  `out` and `lse` are written with plain
+ *     stores only, so they may also be mapped pinned host memory (under
+ *     unified addressing its host address is valid on the device): the
+ *     result then reaches the host without a copy after the call.
  *   - Return value 0 on success, a negative REL_ATTN_ERR_* code otherwise.
  *     Arguments are validated before anything is launched: on an error
  *     nothing runs on the stream.
  *   - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  The caller synchronises.
  *   - One workspace must not be used by two calls that run concurrently.
- *   - Host threads: the library keeps process-wide caches (per-device
- *     attributes, encoded tensor maps, bucket-edge tables) that are not
- *     locked.  Issue calls from one host thread at a time (any number of
- *     streams); callers with several host threads serialise the calls.
+ *   - Host threads: the library keeps process-wide caches (encoded tensor
+ *     maps and bucket-edge tables, behind a mutex; per-device attributes,
+ *     set on first use without one).  Issue calls from one host thread at a
+ *     time (any number of streams); callers with several host threads
+ *     serialise the calls.
  */
 #ifndef REL_ATTN_H
 #define REL_ATTN_H
