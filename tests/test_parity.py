@@ -565,3 +565,27 @@ def test_other_group_sizes_verify_256k(ra, G, T):
     ref = run_oracle(case)
     for splits in (1, 18, 0):
         check(*run_gpu(ra, case, splits), *ref)
+
+
+def test_result_written_into_mapped_host_memory(ra):
+    """out and lse may be mapped pinned host memory (the header allows it):
+    the call then stores the result straight to the host, bit for bit what
+    the same call writes into device memory."""
+    try:
+        from cuda.bindings import runtime as cudart
+    except ImportError:
+        from cuda import cudart
+    case = small(3001, T=2, seed=6)
+    for S in (1, 3):
+        out_d, lse_d = run_gpu(ra, case, S, out_fp32=False)
+        out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+        lse_h = torch.empty(lse_d.shape, dtype=lse_d.dtype).pin_memory()
+        for t in (out_h, lse_h):
+            err, dptr = cudart.cudaHostGetDevicePointer(t.data_ptr(), 0)
+            if int(err) != 0 or int(dptr) != t.data_ptr():
+                pytest.skip("pinned memory is not mapped at its host address")
+        ra.rel_attn_decode(case.q, case.k_cache, case.v_cache, case.block_table, case.seq_lens,
+                           case.rel_table, case.window, S, out=out_h, lse=lse_h,
+                           max_seq_len=case.max_seq_len, out_fp32=False)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
