@@ -12,12 +12,14 @@
 // and likewise for V; the raw (pre-convolution) K/V of every position are
 // kept in a paged sconv cache laid out and addressed like the KV cache.
 //
-// One thread per (new token, KV head, 8 channels): four 16-byte loads of
-// the raw vectors at p, p-1, p-2, p-3 (from the new tokens, or from the
-// sconv cache for positions before them; neighbouring tokens share them
-// through L1), one 64-byte load of the taps, fp32 accumulation with taps in
-// the order 0, 1, 2, 3, then a 16-byte raw store and a 16-byte bf16 (or
-// 8-byte E4M3) cache store.  Positions written (the new ones) and positions
+// One thread per (new token, KV head, 8 channels): eight 16-byte loads of
+// the raw K and V vectors at p, p-1, p-2, p-3 (from the new tokens, or from
+// the sconv cache for positions before them; neighbouring tokens share them
+// through L1), all issued before any arithmetic (K then V one at a time
+// measured 37.0 against 34.3 us for 8,192 tokens, 12.1 against 8.2 us for
+// one), a 64-byte load of each tap set, fp32 accumulation with taps in the
+// order 0, 1, 2, 3, then a 16-byte raw store and a 16-byte bf16 (or 8-byte
+// E4M3) cache store per K and V.  Positions written (the new ones) and positions
 // read from the sconv cache (the older ones) never meet, so a launch has no
 // read-after-write hazard of its own.  HBM-bound: per new token and KV head
 // 256 B in, 256 B raw out, 256 B (or 128 B) cache out.
@@ -98,17 +100,12 @@ rel_attn_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
     return;
   }
   const size_t dst = (((size_t)qpage[0] * p.Hkv + h) * kPage + pos % kPage) * kHeadDim + c0;
+  // all eight raw vectors (K and V at pos, pos-1, pos-2, pos-3) first
+  uint4 xs[2][4];
 #pragma unroll
   for (int kv = 0; kv < 2; ++kv) {
     const __nv_bfloat16* src_new = kv ? p.v_new : p.k_new;
-    __nv_bfloat16* raw = kv ? p.v_raw : p.k_raw;
-    // taps of this thread's 8 channels: w[c][i] at element 4c + i
-    const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (((size_t)kv * p.Hkv + h) * kHeadDim + c0) * 4);
-    float w[32];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) bf16x8_to_f32(__ldg(wp + u), w + 8 * u);
-    float acc[8];
-    uint4 x0 = make_uint4(0, 0, 0, 0);
+    const __nv_bfloat16* raw = kv ? p.v_raw : p.k_raw;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int q = pos - i;
@@ -117,18 +114,28 @@ rel_attn_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
         xv = __ldg(reinterpret_cast<const uint4*>(
             src_new + (((size_t)b * p.T + (q - first_new)) * p.Hkv + h) * kHeadDim + c0));
       } else if (q >= 0) {
-        // an older position: the sconv cache (written by earlier steps;
-        // this launch writes only the new positions)
         xv = *reinterpret_cast<const uint4*>(
             raw + (((size_t)qpage[i] * p.Hkv + h) * kPage + q % kPage) * kHeadDim + c0);
       }
-      if (i == 0) x0 = xv;
+      xs[kv][i] = xv;
+    }
+  }
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    __nv_bfloat16* raw = kv ? p.v_raw : p.k_raw;
+    const uint4* wp = reinterpret_cast<const uint4*>(p.conv_w + (((size_t)kv * p.Hkv + h) * kHeadDim + c0) * 4);
+    float w[32];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) bf16x8_to_f32(__ldg(wp + u), w + 8 * u);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
       float x[8];
-      bf16x8_to_f32(xv, x);
+      bf16x8_to_f32(xs[kv][i], x);
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = (i == 0) ? w[4 * c] * x[c] : fmaf(w[4 * c + i], x[c], acc[c]);
     }
-    *reinterpret_cast<uint4*>(raw + dst) = x0;
+    *reinterpret_cast<uint4*>(raw + dst) = xs[kv][0];
     if constexpr (!E4M3) {
       uint4 o;
       __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
