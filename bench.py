@@ -64,6 +64,15 @@ def parse_args():
     return ap.parse_args()
 
 
+def partial_kernel_name(e4m3: bool, q_tokens: int) -> str:
+    """The partial kernel a decode call launches: over an E4M3 cache, up to
+    three tokens run the FP8 kernel (one-token chunks), four and more the
+    multi-token kernel with the codes widened to bf16 in shared memory."""
+    if e4m3 and q_tokens <= 3:
+        return "rel_attn_partial_fp8_kernel"
+    return "rel_attn_partial_kernel (E4M3 codes widened)" if e4m3 else "rel_attn_partial_kernel"
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -478,7 +487,9 @@ def run_ours(args, rank, world, local_rank):
             "us_partial_kernel": round(mean_part * 1e3, 2),
             "us_combine_kernel_after_event": round(statistics.fmean(t_comb) * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if not e4m3 else "bf16 q, e4m3 kv (e4m3 tensor-core MMAs)",
+            "dtype": "bf16" if not e4m3 else (
+                "bf16 q, e4m3 kv (e4m3 tensor-core MMAs)" if case.q_tokens <= 3 else
+                "bf16 q, e4m3 kv (widened to bf16 in shared memory, bf16 tensor-core MMAs)"),
             "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) relative table)" +
                     ("; K/V quantised to E4M3 with per-KV-head amax/448 scales" if e4m3 else ""),
             "config": {"workload": args.workload, "kv_dtype": args.kv_dtype,
@@ -494,7 +505,7 @@ def run_ours(args, rank, world, local_rank):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                          else "fallback 6.65 TB/s",
-                         "kernel": "rel_attn_partial_fp8_kernel" if e4m3 else "rel_attn_partial_kernel",
+                         "kernel": partial_kernel_name(e4m3, case.q_tokens),
                          "traffic": load_traffic(src_hash, args.workload + ("_e4m3" if e4m3 else "")),
                          "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
                          "frac_per_call": round(value / world / peak, 4),

@@ -164,15 +164,26 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
  *                     head h is e4m3(k_code) * k_scale[h], likewise for V.
  * Every other argument, the workspace and the outputs are as for
  * rel_attn_decode / rel_attn_partial (rel_attn_combine merges the splits of
- * either).  The E4M3 tiles go to the tensor cores as they are (E4M3 x E4M3
- * MMAs, fp32 accumulation): the query is carried as two E4M3 terms scaled
- * per row by a power of two (exact for a bf16 query), the softmax weights
- * as three (12 significant bits); the relative term stays bf16.
- * Several query tokens (a verify step, q_tokens 2..9) run as one-token chunks
- * of each sequence, token t attending to the keys before position L - T + t
- * + 1 as in rel_attn_decode; the chunks of one (split, KV head) are launched
- * side by side so that their page reads meet in L2, but each does the
- * one-token work, so T tokens cost about T one-token calls of compute.
+ * either).  Token t of T attends to the keys before position L - T + t + 1
+ * as in rel_attn_decode.  Two kernels serve the call:
+ *   q_tokens 1..3  The E4M3 tiles go to the tensor cores as they are (E4M3 x
+ *                  E4M3 MMAs, fp32 accumulation): the query is carried as
+ *                  two E4M3 terms scaled per row by a power of two (exact
+ *                  for a bf16 query), the softmax weights as three (12
+ *                  significant bits); the relative term stays bf16.  Two or
+ *                  three tokens run as one-token chunks of each sequence in
+ *                  one launch (the chunks of one split and KV head side by
+ *                  side, so that their page reads meet in L2).
+ *   q_tokens 4..9  The multi-token kernel of rel_attn_decode with the codes
+ *                  widened to bf16 in shared memory (exactly: every E4M3
+ *                  value is a bf16 value), k_scale[h] folded into the logit
+ *                  multiplier and v_scale[h] into the final normalisation;
+ *                  with unit scales the result is bit for bit that of
+ *                  rel_attn_decode on the codes' values.  The NaN codes read
+ *                  as +-480 on this path (a saturating quantiser, such as
+ *                  rel_attn_kv_write, never writes them).
+ * The bucket-density limit (see the top of this file) applies with T = 1 for
+ * up to three tokens and with T itself from four on.
  * Limits: Hq/Hkv must be 4, 6 or 8 and the shape valid for rel_attn_decode
  * (else REL_ATTN_ERR_INVALID_ARG).
  */
@@ -345,10 +356,10 @@ int rel_attn_bucket(const rel_attn_shape* shape, int distance);
 int rel_attn_split_pages(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
                          int split, int* first_page, int* end_page);
 
-/* The same for the E4M3 kernel (rel_attn_decode_e4m3 / rel_attn_partial_e4m3),
- * whose partition weighs an exact-range page more: such a tile also reads a
- * 32 KB bf16 relative-row chunk, twice its E4M3 K and V bytes.  Arguments,
- * results and errors as rel_attn_split_pages. */
+/* The same for calls over an E4M3 cache (rel_attn_decode_e4m3 /
+ * rel_attn_partial_e4m3), whose partition weighs an exact-range page more:
+ * such a tile also reads a 32 KB bf16 relative-row chunk, twice its E4M3 K
+ * and V bytes.  Arguments, results and errors as rel_attn_split_pages. */
 int rel_attn_split_pages_e4m3(const rel_attn_shape* shape, int seq_len, int window, int num_splits,
                               int split, int* first_page, int* end_page);
 

@@ -34,6 +34,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   bool attr_set[3][kMaxQTokens] = {};     // [G = 4, 6, 8][T - 1]
+  bool attr_set_f8[3][kMaxQTokens] = {};  // the same, E4M3 cache (T >= 2)
   bool attr_fp8[3] = {};                   // [G = 4, 6, 8]
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -59,6 +60,16 @@ bool encode_fn_ready() {
 // GQA group sizes with kernel instances: 48/8 heads (Inkling 2 Small, every
 // layer) and the 64/8 full / 64/16 sliding layers of the previous Inkling.
 bool group_supported(int G) { return G == 4 || G == 6 || G == 8; }
+
+// E4M3 cache, T query tokens: up to three run as T one-token chunks of the
+// FP8 kernel (E4M3 tensor-core MMAs), four and more through the multi-token
+// kernel with the codes widened to bf16 in shared memory.  Measured on B200
+// (256K-key verify step, 48/8 heads, us per call, chunks / widened): 2 tokens
+// 167 / 282, 3: 244 / 323, 4: 320 / 320, 5: 396 / 364, 6: 472 / 337, 8: 624 /
+// 359, 9: 701 / 419; 32 sequences of 16K-128K keys with 4 tokens 2,921 /
+// 2,860, with 8 tokens 5,790 / 3,237.
+constexpr int kE4m3WidenMinTokens = 4;
+bool e4m3_widened(int q_tokens) { return q_tokens >= kE4m3WidenMinTokens; }
 
 int validate_shape(const rel_attn_shape* s) {
   if (!s) return REL_ATTN_ERR_INVALID_ARG;
@@ -351,17 +362,17 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
   return true;
 }
 
-template <int G, int T>
+template <int G, int T, bool F8>
 int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
   constexpr int N = group_width_for(G, T);
-  if constexpr (N == 0) {
+  if constexpr (N == 0 || (F8 && T == 1)) {
     return REL_ATTN_ERR_INVALID_ARG;                  // no instance for this shape
   } else {
     constexpr int NG = softmax_groups(G, T);
-    using KC = KernelConfig<N, NG, G, T>;
-    auto kern = rel_attn_partial_kernel<N, G, NG, T>;
+    using KC = KernelConfig<N, NG, G, T, F8>;
+    auto kern = rel_attn_partial_kernel<N, G, NG, T, F8>;
     constexpr int smem = KC::kAllocBytes;
-    bool& attr = di.attr_set[G / 2 - 2][T - 1];
+    bool& attr = F8 ? di.attr_set_f8[G / 2 - 2][T - 1] : di.attr_set[G / 2 - 2][T - 1];
     if (!attr) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return REL_ATTN_ERR_CUDA;
@@ -373,19 +384,19 @@ int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t 
   }
 }
 
-template <int G>
+template <int G, bool F8>
 int launch_partial_group(const DecodeParams& prm, int T, int S, int B, int Hkv, cudaStream_t st,
                          DeviceInfo& di) {
   switch (T) {
-    case 1: return launch_partial<G, 1>(prm, S, B, Hkv, st, di);
-    case 2: return launch_partial<G, 2>(prm, S, B, Hkv, st, di);
-    case 3: return launch_partial<G, 3>(prm, S, B, Hkv, st, di);
-    case 4: return launch_partial<G, 4>(prm, S, B, Hkv, st, di);
-    case 5: return launch_partial<G, 5>(prm, S, B, Hkv, st, di);
-    case 6: return launch_partial<G, 6>(prm, S, B, Hkv, st, di);
-    case 7: return launch_partial<G, 7>(prm, S, B, Hkv, st, di);
-    case 8: return launch_partial<G, 8>(prm, S, B, Hkv, st, di);
-    case 9: return launch_partial<G, 9>(prm, S, B, Hkv, st, di);
+    case 1: return launch_partial<G, 1, F8>(prm, S, B, Hkv, st, di);
+    case 2: return launch_partial<G, 2, F8>(prm, S, B, Hkv, st, di);
+    case 3: return launch_partial<G, 3, F8>(prm, S, B, Hkv, st, di);
+    case 4: return launch_partial<G, 4, F8>(prm, S, B, Hkv, st, di);
+    case 5: return launch_partial<G, 5, F8>(prm, S, B, Hkv, st, di);
+    case 6: return launch_partial<G, 6, F8>(prm, S, B, Hkv, st, di);
+    case 7: return launch_partial<G, 7, F8>(prm, S, B, Hkv, st, di);
+    case 8: return launch_partial<G, 8, F8>(prm, S, B, Hkv, st, di);
+    case 9: return launch_partial<G, 9, F8>(prm, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }
@@ -509,7 +520,9 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   // ---- validation (no CUDA call before this block passes)
   int rc = validate_shape(shape);
   if (rc != REL_ATTN_OK) return rc;
-  if (!bucket_span_fits(shape, kv_e4m3 ? 1 : shape->q_tokens)) return REL_ATTN_ERR_INVALID_ARG;
+  // (one-token chunks need the one-token span)
+  const bool e4m3_chunks = kv_e4m3 && shape->q_tokens > 1 && !e4m3_widened(shape->q_tokens);
+  if (!bucket_span_fits(shape, e4m3_chunks ? 1 : shape->q_tokens)) return REL_ATTN_ERR_INVALID_ARG;
   if (kv_e4m3) {
     if (!k_scale || !v_scale ||
         (reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3))
@@ -539,7 +552,7 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   const uint64_t kv_rows = (uint64_t)shape->num_pages * Hkv * kPage;
   if (!cached_map(&prm->tmap_k, kv_e4m3 ? 4 : 0, k_cache, kv_rows, 0) ||
       !cached_map(&prm->tmap_v, kv_e4m3 ? 5 : 1, v_cache, kv_rows, 0) ||
-      !cached_map(&prm->tmap_r, (kv_e4m3 || group_width_for(Hq / Hkv, T) == 16) ? 3 : 2, rel_table,
+      !cached_map(&prm->tmap_r, group_width_for(Hq / Hkv, e4m3_chunks ? 1 : T) == 16 ? 3 : 2, rel_table,
                   (uint64_t)shape->num_buckets, (uint64_t)Hkv))
     return REL_ATTN_ERR_CUDA;
   prm->q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -555,9 +568,9 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   prm->timeout_ns = wl ? wl : kDefaultTimeoutNs;
   prm->B = B; prm->T = T; prm->Hq = Hq; prm->Hkv = Hkv;
   prm->cps = 1; prm->seq_stride = T; prm->tok_off = 0; prm->len_off = 0;
-  if (kv_e4m3 && T > 1) {
-    // the E4M3 kernel is a one-token kernel: T tokens run as T one-token
-    // chunks of the sequence, each attending causally up to its position
+  if (e4m3_chunks) {
+    // T one-token chunks of the sequence in one launch, each attending
+    // causally up to its own position
     prm->T = 1;
     prm->cps = T;
   }
@@ -578,13 +591,18 @@ int prepare(const rel_attn_shape* shape, const void* q, const void* k_cache, con
   return REL_ATTN_OK;
 }
 
+// bf16 cache, any token count; with e4m3 set, the E4M3 multi-token instances
+// (T >= 2)
 int launch_partial_any(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
-                       DeviceInfo& di) {
+                       DeviceInfo& di, bool e4m3 = false) {
   const int B = shape->batch, Hkv = shape->num_kv_heads, T = shape->q_tokens;
   switch (shape->num_q_heads / Hkv) {
-    case 4: return launch_partial_group<4>(prm, T, S, B, Hkv, st, di);
-    case 6: return launch_partial_group<6>(prm, T, S, B, Hkv, st, di);
-    case 8: return launch_partial_group<8>(prm, T, S, B, Hkv, st, di);
+    case 4: return e4m3 ? launch_partial_group<4, true>(prm, T, S, B, Hkv, st, di)
+                        : launch_partial_group<4, false>(prm, T, S, B, Hkv, st, di);
+    case 6: return e4m3 ? launch_partial_group<6, true>(prm, T, S, B, Hkv, st, di)
+                        : launch_partial_group<6, false>(prm, T, S, B, Hkv, st, di);
+    case 8: return e4m3 ? launch_partial_group<8, true>(prm, T, S, B, Hkv, st, di)
+                        : launch_partial_group<8, false>(prm, T, S, B, Hkv, st, di);
     default: return REL_ATTN_ERR_INVALID_ARG;
   }
 }
@@ -608,6 +626,7 @@ int launch_partial_e4m3_g(const DecodeParams& prm, int S, int B, int Hkv, cudaSt
 int launch_partial_e4m3(const DecodeParams& prm, const rel_attn_shape* shape, int S, cudaStream_t st,
                         DeviceInfo& di) {
   const int B = shape->batch, Hkv = shape->num_kv_heads;
+  if (e4m3_widened(shape->q_tokens)) return launch_partial_any(prm, shape, S, st, di, true);
   switch (shape->num_q_heads / Hkv) {
     case 4: return launch_partial_e4m3_g<4>(prm, S, B, Hkv, st, di);
     case 6: return launch_partial_e4m3_g<6>(prm, S, B, Hkv, st, di);

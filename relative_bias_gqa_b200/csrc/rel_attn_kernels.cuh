@@ -126,11 +126,12 @@ __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / 
 
 // Compile-time configuration of one kernel instance: N = padded group width
 // (G heads x T tokens rounded up to the MMA N step), NG = softmax groups,
-// G = query heads per KV head, T = query tokens.
+// G = query heads per KV head, T = query tokens, F8 = the KV cache holds E4M3
+// codes (widened to bf16 in shared memory by the softmax warps).
 // K tiles and relative-row chunks share one ring of slots (each slot is
 // released as soon as its MMA has read it); V tiles have their own, deeper
 // ring (a V slot is held until the P.V product of its tile).
-template <int N, int NG, int G, int T>
+template <int N, int NG, int G, int T, bool F8 = false>
 struct KernelConfig {
   // N = 16 (one token): the softmax groups alternate tiles, each with all the
   // rows.  N = 32 / 48 / 64 (2..9 tokens): every group takes every tile, each
@@ -180,12 +181,15 @@ struct KernelConfig {
   // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s_full[2],
   //           s_empty[2], p_full[2], o_full[2], o_empty[2], x_full[kXTables],
   //           x_empty[kXTables], drain (S issuer), drain (P.V issuer),
-  //           plan_full[kPlanSlots], plan_empty[kPlanSlots]
+  //           plan_full[kPlanSlots], plan_empty[kPlanSlots], and with an
+  //           E4M3 cache kconv[KS] (the slot's item passed by every softmax
+  //           warp: a K tile widened, a relative chunk let by)
   // Tile plans (column-split instances): the producer, which plans every
   // tile for its own loads, hands each plan to the softmax groups through a
   // ring of kPlanSlots records instead of every softmax thread re-planning.
   static constexpr int kPlanSlots = kAlt ? 0 : 4;
-  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 12 + 2 * kXTables + 2 * kPlanSlots;
+  static constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 12 + 2 * kXTables + 2 * kPlanSlots +
+                                  (F8 ? kKSlots : 0);
   // tmem base, abort flag, bad-page flag, K-ring and V-ring items issued
   static constexpr int oMisc = oBar + kNumBars * 8;
   // per K slot: 1 if its item is a relative-row chunk, 0 a K tile (producer
@@ -447,12 +451,106 @@ __device__ void fill_rows(const DecodeParams& p, int tok0, int h, int s, float o
   }
 }
 
+// Two E4M3 codes of w (the bytes `sel` picks, with their sign bytes) as a
+// bf16 pair, exactly.  A code's exponent and mantissa bits, placed in a bf16's
+// exponent-field low bits and mantissa top bits, read as 2^-120 times the
+// code's value (subnormal codes become bf16 subnormals of the same scaled
+// value); one bf16 multiply by 2^120 rebiases.  The NaN codes 0x7f / 0xff
+// read as +-480 (a saturating quantiser never writes them).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
+  uint32_t x, r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(x) : "r"(w), "r"(sel));
+  x = (x << 4) & 0x87f087f0u;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x7b807b80u));
+  return r;
+}
+
+// Widens this warp's share of one tile (128 keys x 128 dims) of E4M3 codes
+// in place into the bf16 layout of a ring slot: two 64-dim halves of 128 rows
+// x 128 B, 16-byte chunks 128B-swizzled.  The codes sit in the upper half,
+// key r's 128 codes in row r (chunk c = dims 16c..16c+15, swizzled the same
+// way).  Key r's dims 0..63 go to the lower half's row r and dims 64..127 to
+// the upper half's row r, which is the key's own code row, so the warp reads
+// whole rows before it writes them.  Warp w of nw takes the 4-row quads w,
+// w + nw, ... (two per pass); lanes 8i..8i+7 take chunks 0..3 of one row and
+// 4..7 of its neighbour (row ^ 1), so that neither the loads nor the stores
+// of a quarter-warp share a bank.  Rows for which zero_row(r) holds are
+// written as zeros.
+template <class ZeroRow>
+__device__ __forceinline__ void widen_e4m3_rows(uint8_t* slot, int w, int nw, int lane,
+                                                ZeroRow zero_row) {
+  const int c = lane & 7;
+  const int rr = (lane >> 3) ^ (c >> 2);
+  const uint8_t* src = slot + kHalfTileBytes;
+  uint8_t* dst = slot + (c >> 2) * kHalfTileBytes;
+  const int j0 = 2 * (c & 3);                     // bf16 chunks j0, j0 + 1 of the half row
+  auto ld = [&](int r) {
+    return *reinterpret_cast<const uint4*>(src + r * 128 + ((c ^ (r & 7)) << 4));
+  };
+  auto st = [&](int r, const uint4& in) {
+    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;   // dims 16c..16c+7, 16c+8..16c+15
+    if (!zero_row(r)) {
+      lo.x = e4m3x2_to_bf16x2(in.x, 0x9180u);
+      lo.y = e4m3x2_to_bf16x2(in.x, 0xb3a2u);
+      lo.z = e4m3x2_to_bf16x2(in.y, 0x9180u);
+      lo.w = e4m3x2_to_bf16x2(in.y, 0xb3a2u);
+      hi.x = e4m3x2_to_bf16x2(in.z, 0x9180u);
+      hi.y = e4m3x2_to_bf16x2(in.z, 0xb3a2u);
+      hi.z = e4m3x2_to_bf16x2(in.w, 0x9180u);
+      hi.w = e4m3x2_to_bf16x2(in.w, 0xb3a2u);
+    }
+    *reinterpret_cast<uint4*>(dst + r * 128 + ((j0 ^ (r & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(dst + r * 128 + (((j0 + 1) ^ (r & 7)) << 4)) = hi;
+  };
+  constexpr int kQuads = kTileKeys / 4;
+#pragma unroll 1
+  for (int qd = w; qd < kQuads; qd += 2 * nw) {
+    const int r1 = 4 * qd + rr, r2 = 4 * (qd + nw) + rr;
+    const bool two = qd + nw < kQuads;             // the same for the whole warp
+    const uint4 in1 = ld(r1);
+    const uint4 in2 = two ? ld(r2) : in1;
+    __syncwarp();
+    st(r1, in1);
+    if (two) st(r2, in2);
+    __syncwarp();
+  }
+}
+
+// E4M3 cache: the softmax warps pass the K-ring items on in order (kc counts
+// them): a relative-row chunk is let by, a K tile widened (each warp its
+// share of the rows), and every warp's pass is counted on the slot's kconv
+// barrier.  Passes items until one K tile has been passed (returns 1); with
+// `block` false it returns 0 at the first item whose copy has not landed
+// (the next call resumes there); -1 when a wait gave up.
+template <int KS, int kSlotBytes>
+__device__ __forceinline__ int f8_pass_k(int& kc, bool block, uint32_t kfull0, uint32_t kconv0,
+                                         const uint8_t* item_flag, uint8_t* kring, int w, int nw,
+                                         int lane, volatile int* abort_flag,
+                                         unsigned long long tlim) {
+  while (true) {
+    const uint32_t fb = kfull0 + 8u * (uint32_t)(kc % KS);
+    const uint32_t par = (uint32_t)(kc / KS) & 1u;
+    if (block) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(fb, par, abort_flag, tlim))) return -1;
+    } else if (!__all_sync(0xffffffffu, ptx::mbar_test_wait(fb, par))) {
+      return 0;
+    }
+    const bool chunk = item_flag[kc % KS] != 0;
+    if (!chunk) widen_e4m3_rows(kring + (kc % KS) * kSlotBytes, w, nw, lane, [](int) { return false; });
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(kconv0 + 8u * (uint32_t)(kc % KS));
+    ++kc;
+    if (!chunk) return 1;
+  }
+}
+
 // T (query tokens) is a template parameter: every per-row loop below runs
 // over the NQ = T*G live rows only, fully unrolled.
-template <int N, int G, int NG, int T>
-__global__ void __launch_bounds__(KernelConfig<N, NG, G, T>::kThreads, 1)
+template <int N, int G, int NG, int T, bool F8 = false>
+__global__ void __launch_bounds__(KernelConfig<N, NG, G, T, F8>::kThreads, 1)
 rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
-  using KC = KernelConfig<N, NG, G, T>;
+  using KC = KernelConfig<N, NG, G, T, F8>;
   constexpr int KS = KC::kKSlots;
   constexpr int VS = KC::kVSlots;
   constexpr int ROWS = KC::kRows;
@@ -530,6 +628,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const uint32_t drain_pv = drain_bar + 8u;
   auto plan_full = [&](int s) { return drain_pv + 8u * (1 + s); };
   auto plan_empty = [&](int s) { return drain_pv + 8u * (1 + KC::kPlanSlots + s); };
+  auto kconv = [&](int s) { return drain_pv + 8u * (1 + 2 * KC::kPlanSlots + s); };
   uint8_t* item_flag = smem + KC::oItemFlag;
   int4* plan_rec = reinterpret_cast<int4*>(smem + KC::oPlan);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + KC::oMisc);
@@ -541,18 +640,17 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   const unsigned long long tlim = p.timeout_ns;
 
   // -------------------------------------------------------------- prologue
-  // Barriers first, one per lane of warp 0 (in index order: the rings' full /
+  // Barriers first, by the lanes of warp 0 (in index order: the rings' full /
   // empty pairs, s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2],
-  // x_full[X], x_empty[X], the two drains, plan_full / plan_empty[kPlanSlots];
-  // arrival counts 1, or one per
-  // consumer thread for the barriers the softmax threads arrive on).  The
+  // x_full[X], x_empty[X], the two drains, plan_full / plan_empty[kPlanSlots],
+  // then kconv[KS]; arrival counts 1, one per consumer thread for the
+  // barriers the softmax threads arrive on, one per softmax warp for kconv).  The
   // producer's first block-table entries are requested before the CTA-wide
   // barrier; the other warps then allocate tensor memory and stage Q and the
   // bucket edges.
-  static_assert(KC::kNumBars <= 32, "one barrier per lane");
   if (warp == 0) {
-    if (lane < KC::kNumBars) {
-      const int r = lane - kB;
+    auto init_bar = [&](int i) {
+      const int r = i - kB;
       const uint32_t cnt =
           (r < 0) ? 1u
           : (r < 2) ? 1u                                      // s_full
@@ -562,10 +660,16 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           : (r < 10 + KC::kXTables) ? 1u                      // x_full
           : (r < 10 + 2 * KC::kXTables) ? (uint32_t)KC::kConsumers   // x_empty
           : (r < 12 + 2 * KC::kXTables + KC::kPlanSlots) ? 1u        // drains, plan_full
-          : (uint32_t)KC::kConsumers;                         // plan_empty
-      ptx::mbar_init(bar0 + 8u * lane, cnt);
-      ptx::fence_mbar_init();
+          : (r < 12 + 2 * KC::kXTables + 2 * KC::kPlanSlots) ? (uint32_t)KC::kConsumers  // plan_empty
+          : (uint32_t)(KC::kConsumers / 32);                  // kconv
+      ptx::mbar_init(bar0 + 8u * i, cnt);
+    };
+    if constexpr (KC::kNumBars <= 32) {
+      if (lane < KC::kNumBars) init_bar(lane);
+    } else {
+      for (int i = lane; i < KC::kNumBars; i += 32) init_bar(i);
     }
+    ptx::fence_mbar_init();
     if (lane == 0) {
       *abort_flag = 0;
       *bad_page_flag = 0;
@@ -687,11 +791,21 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           const uint32_t st = kslot(k);
           const uint32_t fb = kfull(k % KS);
           item_flag[k % KS] = 0;
-          ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
-          for (int pi = 0; pi < tp.npg; ++pi) {
-            const int row = pi ? rows1[ti & 1] : rows0[ti & 1];
-            ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
-            ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
+          if constexpr (F8) {
+            // E4M3 codes, one 128-byte row per key, into the slot's upper
+            // half (where the widened dims 64..127 of the same key go)
+            ptx::mbar_arrive_expect_tx(fb, tp.npg * kPageHalfBytes);
+            for (int pi = 0; pi < tp.npg; ++pi) {
+              const int row = pi ? rows1[ti & 1] : rows0[ti & 1];
+              ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
+            }
+          } else {
+            ptx::mbar_arrive_expect_tx(fb, tp.npg * 2 * kPageHalfBytes);
+            for (int pi = 0; pi < tp.npg; ++pi) {
+              const int row = pi ? rows1[ti & 1] : rows0[ti & 1];
+              ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_k, fb, 0, row, pol);
+              ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_k, fb, 64, row, pol);
+            }
           }
         }
         ++k;
@@ -705,11 +819,19 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
         if (lane == 0) {
           const uint32_t st = vslot(tv);
           const uint32_t fb = vfull(tv % VS);
-          ptx::mbar_arrive_expect_tx(fb, npgs[tv & 1] * 2 * kPageHalfBytes);
-          for (int pi = 0; pi < npgs[tv & 1]; ++pi) {
-            const int row = pi ? rows1[tv & 1] : rows0[tv & 1];
-            ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
-            ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
+          if constexpr (F8) {
+            ptx::mbar_arrive_expect_tx(fb, npgs[tv & 1] * kPageHalfBytes);
+            for (int pi = 0; pi < npgs[tv & 1]; ++pi) {
+              const int row = pi ? rows1[tv & 1] : rows0[tv & 1];
+              ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
+            }
+          } else {
+            ptx::mbar_arrive_expect_tx(fb, npgs[tv & 1] * 2 * kPageHalfBytes);
+            for (int pi = 0; pi < npgs[tv & 1]; ++pi) {
+              const int row = pi ? rows1[tv & 1] : rows0[tv & 1];
+              ptx::tma_load_2d(st + pi * kPageHalfBytes, &p.tmap_v, fb, 0, row, pol);
+              ptx::tma_load_2d(st + kHalfTileBytes + pi * kPageHalfBytes, &p.tmap_v, fb, 64, row, pol);
+            }
           }
         }
         i_v = tv + 1;
@@ -734,9 +856,15 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       const uint64_t qdesc0 = ptx::sdesc_sw128(sQ, 16, 1024);                      // Q, K-major
       int k = 0;                               // K-ring items taken
       int cg[2] = {0, 0};                      // chunks issued per group
+      // an item is ready once its copy has landed and, with an E4M3 cache,
+      // every softmax warp has passed it (widened a K tile, or let a chunk by)
+      auto k_ready = [&](int kk) {
+        return ptx::mbar_wait(kfull(kk % KS), (kk / KS) & 1, abort_flag, tlim) &&
+               (!F8 || ptx::mbar_wait(kconv(kk % KS), (kk / KS) & 1, abort_flag, tlim));
+      };
       for (int ti = 0; ti < g.ntiles; ++ti) {
         const int gq = KC::kAlt ? (ti & 1) : 0;
-        if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
+        if (!k_ready(k)) break;
         if (item_flag[k % KS]) {
           // the tile's new relative-row chunk came first: X = R_chunk . Q
           const int c = cg[gq];
@@ -755,7 +883,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           ptx::umma_commit(kempty(k % KS));
           ++k;
           cg[gq] = c + 1;
-          if (!ptx::mbar_wait(kfull(k % KS), (k / KS) & 1, abort_flag, tlim)) break;
+          if (!k_ready(k)) break;
         }
         if (!ptx::mbar_wait(s_empty + 8u * (ti & 1), ((ti >> 1) & 1) ^ 1, abort_flag, tlim)) break;
         ptx::tc_fence_after();
@@ -864,7 +992,23 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     for (int r = 0; r < (KC::kAlt ? RG : 1); ++r) alpha_r[r] = 1.f;
     int c = 0, li = 0;                        // own chunks, own tiles
     PlanState ps(p.nl);                       // planned over this group's tiles
+    // E4M3 cache: multiplier of the K.Q product with the K scale folded in
+    // (the relative term is not scaled by it)
+    float s_mul_f8 = 0.f;
+    if constexpr (F8) s_mul_f8 = p.scale_log2 * __ldg(p.k_scale + h);
     bool failed = false, aborted = false;
+    // E4M3 cache: K-ring items this warp has passed on, K tiles among them.
+    // Tile t + 1's K is passed at the start of tile t if its copy has landed
+    // (its S product then runs during tile t's softmax), else right after
+    // tile t's P is handed on; tile t's V is widened just before that.
+    int kc = 0, k_passed = 0;
+    if constexpr (F8) {
+      if (f8_pass_k<KS, KC::kKSlotBytes>(kc, true, kfull(0), kconv(0), item_flag, smem + KC::oK, warp - 2,
+                                         4 * NG, lane, abort_flag, tlim) < 0)
+        failed = true;
+      else
+        k_passed = 1;
+    }
 
     // Accumulate the O^T tile of tile j (this thread's head-dim lane, this
     // group's columns) with the rescale factors `al` of that tile.
@@ -912,6 +1056,12 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
     for (int ti = t_first; ti < g.ntiles; ti += kStep) {
       TilePlan tp = tp_next;
       int c0 = c0_next;
+      if constexpr (F8) {
+        if (k_passed == ti + 1 && ti + 1 < g.ntiles &&
+            f8_pass_k<KS, KC::kKSlotBytes>(kc, false, kfull(0), kconv(0), item_flag, smem + KC::oK,
+                                           warp - 2, 4 * NG, lane, abort_flag, tlim) > 0)
+          ++k_passed;
+      }
       if constexpr (KC::kPlanSlots > 0) {
         // the producer's plan of this tile (all threads of the group agree on
         // whether it arrived before any of them acts on it)
@@ -994,7 +1144,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
           const int r = tt * G + gg;
-          s[r] = v ? fmaf(s[r], p.scale_log2, yrow[r]) : -INFINITY;
+          s[r] = v ? fmaf(s[r], F8 ? s_mul_f8 : p.scale_log2, yrow[r]) : -INFINITY;
         }
       }
       // ---- lazy max: p = exp2(x - m_ref) with the row's reference max
@@ -1089,8 +1239,19 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       }
       // ---- keys no token may see: clear their V rows (stale or poisoned data
       //      must not reach the P.V product, where 0 * NaN = NaN); with both
-      //      groups on the tile, group 0 does it
-      if (KC::kAlt || grp == 0) {
+      //      groups on the tile, group 0 does it.  E4M3 cache: every softmax
+      //      warp widens its share of the V tile, writing those rows as zeros.
+      if constexpr (F8) {
+        if (__all_sync(0xffffffffu, ptx::mbar_wait(vfull(i % VS), (i / VS) & 1, abort_flag, tlim))) {
+          const int jt = tp.j0, nload = tp.npg * kPage;
+          widen_e4m3_rows(smem + KC::oV + (i % VS) * kVSlotBytes, warp - 2, 4 * NG, lane, [&](int r) {
+            const int jr = jt + r;
+            return !(r < nload && jr <= g.L - 1 && (g.W <= 0 || g.p0 - jr < g.W));
+          });
+        } else {
+          failed = true;
+        }
+      } else if (KC::kAlt || grp == 0) {
         const bool any_valid = loaded && j <= g.L - 1 && (g.W <= 0 || g.p0 - j < g.W);
         if (!any_valid) {
           // The row is cleared after its copy has landed.  If the wait gives
@@ -1110,6 +1271,16 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(p_full + 8u * (i & 1));
+      if constexpr (F8) {
+        // (skipped by the whole warp once any lane has given up a wait)
+        if (k_passed == ti + 1 && ti + 1 < g.ntiles && !__any_sync(0xffffffffu, failed)) {
+          if (f8_pass_k<KS, KC::kKSlotBytes>(kc, true, kfull(0), kconv(0), item_flag, smem + KC::oK,
+                                             warp - 2, 4 * NG, lane, abort_flag, tlim) < 0)
+            failed = true;
+          else
+            ++k_passed;
+        }
+      }
       if (KC::kAlt && ti + kStep < g.ntiles) {
         tp_next = plan_tile<ROWS>(g, ti + kStep, p.ex, p.log2_ex, p.log_scale, s_edges, ps);
         c0_next = ps.c0;
@@ -1197,6 +1368,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
           l = es[idx];
         }
         o = (l > 0.f) ? o / l : 0.f;
+        if constexpr (F8) o *= __ldg(p.v_scale + h);
         const float lse_v = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
         const int row = (row0 + t) * p.Hq + h * G + gg;
         if (p.num_splits == 1) {

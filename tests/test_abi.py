@@ -297,6 +297,26 @@ def test_bucket_tables_too_dense_for_a_chunk_are_rejected(ra, nb, e, dmax, T):
         assert rc == ra.REL_ATTN_ERR_NO_DEVICE
 
 
+@pytest.mark.parametrize("nb,e,dmax", EDGE_TRIPLES + [(600, 100, 8000), (350, 100, 1500)],
+                         ids=[str(t) for t in EDGE_TRIPLES + [(600, 100, 8000), (350, 100, 1500)]])
+@pytest.mark.parametrize("T", [2, 3, 4, 8])
+def test_e4m3_span_rule_follows_the_path(ra, nb, e, dmax, T):
+    """Over an E4M3 cache up to three tokens run as one-token chunks (the
+    one-token span rule applies), four and more through the multi-token
+    kernel (the T-token rule)."""
+    s = shape(ra, num_buckets=nb, exact_buckets=e, max_distance=dmax, q_tokens=T,
+              num_q_heads=48, num_kv_heads=8)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = ra.lib.rel_attn_decode_e4m3(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
+                                     fake, 0, 1, fake, None, fake, 1 << 30, None)
+    tt = 1 if T <= 3 else T
+    too_dense = _span_oracle(nb, e, dmax, tt) > (128 if tt == 1 else 136)
+    if too_dense:
+        assert rc == ra.REL_ATTN_ERR_INVALID_ARG
+    elif not torch.cuda.is_available():
+        assert rc == ra.REL_ATTN_ERR_NO_DEVICE
+
+
 def test_dense_table_in_the_edge_tests_is_too_dense(ra):
     assert _span_oracle(600, 100, 1500, 1) > 128 and _span_oracle(600, 100, 1500, 2) > 136
     assert _span_oracle(1280, 1024, 1 << 20, 1) == 128 and _span_oracle(1280, 1024, 1 << 20, 8) == 135

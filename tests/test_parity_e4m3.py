@@ -1,10 +1,13 @@
 """GPU parity of the E4M3 (FP8) KV-cache path against the fp64 oracle.
 
 The oracle dequantises the codes exactly (code value x per-KV-head scale) and
-applies the definition; the kernel runs the codes through E4M3 tensor-core
-MMAs, with the query split into two E4M3 terms and P into three.  Same
-tolerances as the bf16 path: max |out_fp32 - oracle| <= 2e-3, max |lse -
-oracle| <= 1e-3.
+applies the definition.  Up to three query tokens: the FP8 kernel runs the
+codes through E4M3 tensor-core MMAs, with the query split into two E4M3
+terms and P into three (several tokens as one-token chunks of one launch).
+Four and more: the multi-token kernel widens the codes to bf16 in shared
+memory (exactly) and folds the scales into the logit multiplier and the
+final normalisation.  Same tolerances as the bf16 path: max |out_fp32 -
+oracle| <= 2e-3, max |lse - oracle| <= 1e-3.
 """
 
 import numpy as np
@@ -249,7 +252,7 @@ MULTI = [
 @pytest.mark.parametrize("splits", [1, 3, 0])
 def test_several_query_tokens(ra, kw, splits):
     """A verify step over the E4M3 cache: token t of T sees the keys up to
-    position L - T + t (one-token chunks of the same launch)."""
+    position L - T + t."""
     case = small(**kw)
     codes = e4m3(case)
     out, lse = run_gpu(ra, case, codes, splits)
@@ -275,10 +278,70 @@ def test_verify_256k_eight_tokens_one_kv_head(ra):
     check(out, lse, ref_out, ref_lse)
 
 
-def test_several_query_tokens_match_one_token_calls(ra):
-    """Token t of a T-token call equals a one-token call whose sequence ends
-    at that token (same splits: the same chunks, bit for bit)."""
-    T, L = 4, 3001
+def _all_finite_codes(shape, gen):
+    """Uniform E4M3 codes over the 254 finite ones (0x7f and 0xff are NaN):
+    subnormal codes (exponent field 0) and both zeros included."""
+    c = torch.randint(0, 254, shape, generator=gen, dtype=torch.int16)
+    c = c + (c >= 0x7F).to(torch.int16)
+    return c.to(torch.uint8)
+
+
+@pytest.mark.parametrize("kw", [dict(T=4, L=3001), dict(T=5, L=700, window=64),
+                                dict(T=8, L=4000, seed=2), dict(T=9, L=1700, G=4, window=512, NB=1024),
+                                dict(T=6, L=2500, G=8), dict(T=8, L=130, G=8)],
+                         ids=lambda k: str(k))
+def test_several_query_tokens_equal_bf16_on_the_decoded_codes(ra, kw):
+    """With unit scales a multi-token E4M3 call (four tokens or more) equals,
+    bit for bit, the bf16 call on the codes' values (every E4M3 value is a
+    bf16 value): the kernel widens the codes to bf16 in shared memory and
+    then runs the bf16 arithmetic.  Every finite code occurs, subnormal ones included; one
+    split, so that both calls walk the same pages."""
+    case = small(**kw)
+    gen = torch.Generator().manual_seed(11)
+    kc = _all_finite_codes(case.k_cache.shape, gen).to("cuda")
+    vc = _all_finite_codes(case.v_cache.shape, gen).to("cuda")
+    ones = torch.ones(case.k_cache.shape[1], dtype=torch.float32, device="cuda")
+    out8, lse8 = run_gpu(ra, case, (kc, vc, ones, ones), 1)
+    kb = kc.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    vb = vc.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    out16, lse16 = ra.rel_attn_decode(case.q, kb, vb, case.block_table, case.seq_lens,
+                                      case.rel_table, case.window, 1, max_seq_len=case.max_seq_len,
+                                      out_fp32=True, exact_buckets=case.exact_buckets,
+                                      max_distance=case.max_distance)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out8).all()
+    assert torch.equal(out8, out16) and torch.equal(lse8, lse16)
+
+
+def test_several_query_tokens_nan_codes_in_unseen_slots_do_not_matter(ra):
+    """Several tokens over E4M3 NaN codes in every slot no query sees (the
+    widened path and the one-token chunks)."""
+    for kw in (dict(L=3001, T=8), dict(L=2500, T=4, window=1024, NB=1024), dict(L=3001, T=3)):
+        case = small(**kw)
+        kc, vc, ks, vs = e4m3(case)
+        ref = run_oracle(case, (kc, vc, ks, vs))
+        L, T = int(case.seq_lens[0]), kw["T"]
+        lo = max(0, L - T - case.window + 1) if case.window > 0 else 0
+        seen = torch.zeros(kc.shape[0], kc.shape[2], dtype=torch.bool)
+        bt = case.block_table[0].cpu()
+        for j in range(lo, L):
+            seen[int(bt[j // 64]), j % 64] = True
+        mask = (~seen).to(kc.device)[:, None, :, None].expand_as(kc)
+        kp, vp = kc.clone(), vc.clone()
+        kp[mask] = 0x7F
+        vp[mask] = 0xFF
+        for splits in (1, 4):
+            clean = run_gpu(ra, case, (kc, vc, ks, vs), splits)
+            bad = run_gpu(ra, case, (kp, vp, ks, vs), splits)
+            assert torch.equal(clean[0], bad[0]) and torch.equal(clean[1], bad[1])
+            check(*bad, *ref)
+
+
+def test_up_to_three_tokens_match_one_token_calls(ra):
+    """Up to three tokens run as one-token chunks of one launch: token t of
+    a T-token call equals a one-token call whose sequence ends at that token
+    (same splits: the same chunks, bit for bit)."""
+    T, L = 3, 3001
     case = small(L, T=T, seed=9)
     codes = e4m3(case)
     out, lse = run_gpu(ra, case, codes, 3)
