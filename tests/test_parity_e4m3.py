@@ -260,8 +260,11 @@ def test_several_query_tokens(ra, kw, splits):
     check(out, lse, ref_out, ref_lse)
 
 
-def test_several_query_tokens_batched(ra):
-    case = small(0, lens=[9, 130, 2049, 700], T=3, seed=4)
+@pytest.mark.parametrize("T", [3, 6])
+def test_several_query_tokens_batched(ra, T):
+    """Mixed lengths in one batch: three tokens (one-token chunks) and six
+    (codes widened in shared memory)."""
+    case = small(0, lens=[9, 130, 2049, 700], T=T, seed=4)
     codes = e4m3(case)
     out, lse = run_gpu(ra, case, codes, 0)
     ref_out, ref_lse = run_oracle(case, codes)
