@@ -100,8 +100,9 @@ rel_attn_partial_fp8_kernel(const __grid_constant__ DecodeParams p) {
   constexpr float kLazy8 = 8.f;               // P = exp2(x - m_ref) <= 2^8 < 448
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array so that the
+  // compiler keeps every access through smem in the shared window
+  uint8_t* smem = smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = ptx::smem_addr(smem);
 
   const int tid = threadIdx.x;
