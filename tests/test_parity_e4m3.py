@@ -204,11 +204,15 @@ def test_previous_model_full_layer(ra, name):
         check(*run_gpu(ra, case, codes, s), *ref)
 
 
-def test_injected_wait_limit_times_out_cleanly(ra):
-    """As for the bf16 kernel: a 1 ns wait bound makes the E4M3 kernel abort
-    promptly with TIMEOUT and NaN rows; the default bound then works again."""
+@pytest.mark.parametrize("T", [1, 8])
+def test_injected_wait_limit_times_out_cleanly(ra, T):
+    """As for the bf16 kernel: a 1 ns wait bound makes the E4M3 kernels abort
+    promptly with TIMEOUT and NaN rows (one token: the FP8 kernel; eight: the
+    widened multi-token kernel, whose softmax warps also wait for K copies);
+    the default bound then works again."""
     import time
-    case = W.make_workload("full_100k", seed=4, device="cuda", num_q_heads=12, num_kv_heads=2)
+    case = W.make_workload("full_100k", seed=4, device="cuda", num_q_heads=12, num_kv_heads=2,
+                           q_tokens=T)
     codes = e4m3(case)
     shape = ra.shape_of(case.q, codes[0], case.block_table, case.rel_table,
                         max_seq_len=case.max_seq_len, out_fp32=True)
