@@ -106,8 +106,11 @@ def test_split_count_invariance(ra):
         check(*run_gpu(ra, case, codes, s), *ref)
 
 
-def test_bf16_output_is_rounded_fp32(ra):
-    case = small(2600)
+@pytest.mark.parametrize("T", [1, 8])
+def test_bf16_output_is_rounded_fp32(ra, T):
+    """bf16 output is the fp32 output rounded (one token: the FP8 kernel;
+    eight: the widened multi-token kernel)."""
+    case = small(2600, T=T)
     codes = e4m3(case)
     for splits in (1, 4):
         o32, l32 = run_gpu(ra, case, codes, splits, out_fp32=True)
@@ -139,9 +142,11 @@ def test_nan_codes_in_unseen_slots_do_not_matter(ra):
             check(*bad, *ref)
 
 
-def test_scales_are_per_kv_head(ra):
-    """Distinct scales per head: doubling head 1's V scale doubles only its rows."""
-    case = small(3000)
+@pytest.mark.parametrize("T", [1, 8])
+def test_scales_are_per_kv_head(ra, T):
+    """Distinct scales per head: doubling head 1's V scale doubles only its rows
+    (one token, and eight through the widened multi-token kernel)."""
+    case = small(3000, T=T)
     kc, vc, ks, vs = e4m3(case)
     o1, l1 = run_gpu(ra, case, (kc, vc, ks, vs), 3)
     vs2 = vs.clone()
@@ -149,6 +154,7 @@ def test_scales_are_per_kv_head(ra):
     o2, l2 = run_gpu(ra, case, (kc, vc, ks, vs2), 3)
     assert torch.equal(o1[:, :, :6], o2[:, :, :6])
     assert torch.allclose(o2[:, :, 6:], 2 * o1[:, :, 6:], rtol=1e-6, atol=0)
+    check(o2, l2, *run_oracle(case, (kc, vc, ks, vs2)))
     assert torch.equal(l1, l2)
 
 
