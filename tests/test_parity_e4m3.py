@@ -291,6 +291,17 @@ def test_verify_256k_eight_tokens_one_kv_head(ra):
     check(out, lse, ref_out, ref_lse)
 
 
+def test_previous_model_full_layer_eight_tokens_one_kv_head(ra):
+    """The 64/8 full-attention layer (G = 8) at 100K keys with an 8-token
+    verify over E4M3, one KV head: the widened 64-wide four-group instance
+    at full size against the oracle's 8 x 8 rows."""
+    case = small(100_000, T=8, G=8, Hkv=1, seed=11)
+    codes = e4m3(case)
+    out, lse = run_gpu(ra, case, codes, 0)
+    ref_out, ref_lse = run_oracle(case, codes)
+    check(out, lse, ref_out, ref_lse)
+
+
 def _all_finite_codes(shape, gen):
     """Uniform E4M3 codes over the 254 finite ones (0x7f and 0xff are NaN):
     subnormal codes (exponent field 0) and both zeros included."""
