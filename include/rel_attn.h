@@ -179,7 +179,10 @@ int rel_attn_combine(const rel_attn_shape* shape, int num_splits, void* out,
  *                  value is a bf16 value), k_scale[h] folded into the logit
  *                  multiplier and v_scale[h] into the final normalisation;
  *                  with unit scales the result is bit for bit that of
- *                  rel_attn_decode on the codes' values.  The NaN codes read
+ *                  rel_attn_decode on the codes' values for six tokens and
+ *                  more and for five at Hq/Hkv = 8 (at four, and five for
+ *                  Hq/Hkv <= 6, the rows are split over four softmax groups
+ *                  instead of two, which agrees to rounding).  The NaN codes read
  *                  as +-480 on this path (a saturating quantiser, such as
  *                  rel_attn_kv_write, never writes them).
  * The bucket-density limit (see the top of this file) applies with T = 1 for

@@ -364,11 +364,11 @@ bool cached_map(CUtensorMap* out, int kind, const void* base, uint64_t a, uint64
 
 template <int G, int T, bool F8>
 int launch_partial(const DecodeParams& prm, int S, int B, int Hkv, cudaStream_t st, DeviceInfo& di) {
-  constexpr int N = group_width_for(G, T);
+  constexpr int N = group_width_for(G, T, F8);
   if constexpr (N == 0 || (F8 && T == 1)) {
     return REL_ATTN_ERR_INVALID_ARG;                  // no instance for this shape
   } else {
-    constexpr int NG = softmax_groups(G, T);
+    constexpr int NG = softmax_groups(G, T, F8);
     using KC = KernelConfig<N, NG, G, T, F8>;
     auto kern = rel_attn_partial_kernel<N, G, NG, T, F8>;
     constexpr int smem = KC::kAllocBytes;

@@ -58,7 +58,13 @@ constexpr int kBarSetup = 6;                   // every warp but the producer (p
 // S^T (a thread's per-tile work halves and every SM sub-partition runs four
 // softmax warps to hide each other's latencies), and always past 48 query
 // rows (the 64-wide instances); else two.
-__host__ __device__ constexpr int softmax_groups(int G, int T) {
+__host__ __device__ constexpr int softmax_groups(int G, int T, bool f8 = false) {
+  // E4M3 cache (the softmax warps also widen the codes): four groups from
+  // four tokens on spread that work over 16 warps; measured on the 256K
+  // verify step at G = 6, 4 tokens 257 against 298 us, 5 tokens 328 against
+  // 341; 100K keys at G = 8, 4 tokens 119 against 135, but 5 tokens 169
+  // against 158 (that instance spills), so G = 8 keeps two groups there.
+  if (f8 && (T == 4 || (T == 5 && G <= 6))) return 4;
   // Six and nine tokens: three groups of two / three tokens.  On the 256K
   // verify step at G = 6: 221 against 265 us (four groups, 1 / 2 / 1 / 2
   // tokens) and 374 against 501 us (2 / 2 / 2 / 3); on 100K keys at G = 8
@@ -246,10 +252,10 @@ struct ColSplit {
 // group's row block 8-aligned, then (four groups) 64 8-aligned, then the
 // smallest of 32 and 48 that holds them 4-aligned, then 64 4-aligned (past 48
 // rows: G = 6 with 9 tokens).
-__host__ __device__ constexpr int group_width_for(int G, int T) {
+__host__ __device__ constexpr int group_width_for(int G, int T, bool f8 = false) {
   if (G < 1 || G > 8 || T < 1 || T > kMaxQTokens) return 0;
   if (T == 1) return 16;
-  const int NG = softmax_groups(G, T);
+  const int NG = softmax_groups(G, T, f8);
   if (cs_end(T, G, NG, 8) <= 32) return 32;
   if (cs_end(T, G, NG, 8) <= 48) return 48;
   // four groups: 8-aligned blocks in a 64-wide tile beat 4-aligned ones in
@@ -585,7 +591,7 @@ rel_attn_partial_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int RG8 = (RG + 7) / 8;
   constexpr int RGL8 = (kAlign == 8) ? RG8 : (RG + 4 + 7) / 8;   // 8-column loads per row block
   constexpr bool kEvenSplit = KC::kAlt || T % NG == 0;
-  static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(G, T) && CSp::end(kAlign) <= N &&
+  static_assert(KC::kAlt ? (NG == 2 && NQ <= N) : (NG == softmax_groups(G, T, F8) && CSp::end(kAlign) <= N &&
                                                    RG <= KC::kGR), "group width");
 
   // ------------------------------------------------------------ geometry

@@ -17,11 +17,12 @@ PROGRAM = r"""
 #include "rel_attn_kernels.cuh"
 using namespace relattn;
 int main() {
+  for (int f8 = 0; f8 <= 1; ++f8)
   for (int G = 1; G <= 8; ++G) {
     for (int T = 1; T <= 9; ++T) {
-      const int N = group_width_for(G, T), NG = softmax_groups(G, T);
+      const int N = group_width_for(G, T, f8 != 0), NG = softmax_groups(G, T, f8 != 0);
       const int A = (T == 1) ? 8 : (cs_end(T, G, NG, 8) <= N ? 8 : 4);
-      std::printf("%d %d %d %d %d", G, T, N, NG, A);
+      std::printf("%d %d %d %d %d %d", f8, G, T, N, NG, A);
       for (int q = 0; q < NG; ++q)
         std::printf(" %d:%d:%d", cs_tok_begin(T, NG, q), cs_slot(T, G, NG, q, A), cs_rows(T, G, NG, q));
       std::printf("\n");
@@ -46,9 +47,9 @@ def table(tmp_path_factory):
     rows = {}
     for line in out.splitlines():
         f = line.split()
-        G, T, N, NG, A = map(int, f[:5])
-        groups = [tuple(map(int, g.split(":"))) for g in f[5:]]
-        rows[(G, T)] = (N, NG, A, groups)
+        F8, G, T, N, NG, A = map(int, f[:6])
+        groups = [tuple(map(int, g.split(":"))) for g in f[6:]]
+        rows[(G, T) if not F8 else (G, T, "e4m3")] = (N, NG, A, groups)
     return rows
 
 
@@ -114,3 +115,23 @@ def test_column_split_layout(table, G, T):
 def test_one_token_instance(table, G):
     N, NG, A, groups = table[(G, 1)]
     assert N == 16 and NG == 2 and G <= N
+
+
+def test_e4m3_widened_instances(table):
+    """Over an E4M3 cache the softmax warps also widen the codes: four groups
+    at four tokens (and five for G <= 6), 8-aligned; otherwise the bf16
+    instances' layout."""
+    assert [table[(G, 4, "e4m3")][:3] for G in (4, 6, 8)] == [(32, 4, 8)] * 3
+    assert [table[(G, 5, "e4m3")][:3] for G in (4, 6)] == [(32, 4, 8), (48, 4, 8)]
+    assert table[(8, 5, "e4m3")] == table[(8, 5)]
+    for G in (4, 6, 8):
+        for T in (6, 7, 8, 9):
+            assert table[(G, T, "e4m3")] == table[(G, T)]
+    # column-split instances (several tokens): every group has tokens, slots
+    # do not overlap, and the block fits N
+    for (key, (N, NG, A, groups)) in table.items():
+        if len(key) == 3 and N and key[1] >= 2:
+            ends = [slot + rows for (_, slot, rows) in groups]
+            assert all(rows > 0 for (_, _, rows) in groups) and max(ends) <= N, key
+            assert all(groups[i][1] + groups[i][2] <= groups[i + 1][1] for i in range(NG - 1)), key
+
